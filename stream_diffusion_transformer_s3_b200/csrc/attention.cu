@@ -1,0 +1,352 @@
+// Varlen joint attention for sm_100a (head dim 128), flash-style with tcgen05.
+//
+// One CTA computes one (branch, head, 128-row query tile):
+//   O = softmax(Q K^T / sqrt(128)) V over all L_b tokens of its branch segment.
+// There is no mask inside a segment: caption pad tokens are ordinary context
+// ("Z-Image-Turbo port", "The three things that each cost a wrong image", item 3),
+// branches never see each other, and only the columns past the segment end of the
+// last key tile are excluded.
+//
+// Warp roles (192 threads):
+//   warp 0 lane 0 : TMA producer (Q once; K and V tiles in separate 2-deep rings)
+//   warp 1 lane 0 : tcgen05.mma issuer (S = Q K^T into TMEM, O += P V from smem P)
+//   warps 2-5     : softmax, one thread per query row (TMEM lane)
+// TMEM columns: S ping-pong at [0,128) and [128,256), O at [256,384).
+// Online softmax in FP32 with a lazily moved reference max: the running max only
+// moves (and O is rescaled) when a row's max grows by more than 2^8, so the common
+// tile needs no O round trip; P = exp2(s - m_ref) <= 256 stays in bf16 range.
+#include <cstdio>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace zdit {
+
+bool make_tmap_bf16_2d(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint64_t ld_elems,
+                       uint32_t box_rows, uint32_t box_cols);
+
+namespace {
+
+constexpr int TILE = 128;          // query rows and key rows per tile
+constexpr int HD = 128;            // head dim
+constexpr int HALF = TILE * 64 * 2;  // one 64-column swizzled half tile: 16 KB
+constexpr int TILE_BYTES = 2 * HALF;
+constexpr int THREADS = 192;
+constexpr int KV_STAGES = 2;
+// smem: Q | K[2] | V[2] | P, then barriers
+constexpr int OFF_Q = 0;
+constexpr int OFF_K = OFF_Q + TILE_BYTES;
+constexpr int OFF_V = OFF_K + KV_STAGES * TILE_BYTES;
+constexpr int OFF_P = OFF_V + KV_STAGES * TILE_BYTES;
+constexpr int OFF_BAR = OFF_P + TILE_BYTES;
+constexpr int SMEM_BYTES = 1024 + OFF_BAR + 256;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+struct AParams {
+  int ldo, n_heads, batch;
+  void* o;
+  const int* cu;
+  float scale_log2;
+  int* err;
+};
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const AParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;   // [2]
+  uint64_t* k_empty = bars + 3;  // [2]
+  uint64_t* v_full = bars + 5;   // [2]
+  uint64_t* v_empty = bars + 7;  // [2]
+  uint64_t* s_full = bars + 9;   // [2]
+  uint64_t* s_empty = bars + 11; // [2]
+  uint64_t* p_full = bars + 13;
+  uint64_t* pv_done = bars + 14;
+  uint64_t* mma_done = bars + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int head = blockIdx.y;
+
+  // locate (branch, query tile) of this CTA
+  int b = 0, qt = blockIdx.x;
+  int seg0 = 0, L = 0;
+  for (; b < p.batch; ++b) {
+    seg0 = p.cu[b];
+    L = p.cu[b + 1] - seg0;
+    const int nq = (L + TILE - 1) / TILE;
+    if (qt < nq) break;
+    qt -= nq;
+  }
+  if (b >= p.batch) return;  // (grid sized exactly; defensive, uniform per CTA)
+  const int n_kv = (L + TILE - 1) / TILE;
+  const int q0 = seg0 + qt * TILE;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], 4);
+    }
+    mbar_init(p_full, 4);
+    mbar_init(pv_done, 1);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int col0 = head * HD;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ producer
+    uint8_t* sQ = smem + OFF_Q;
+    mbar_arrive_expect_tx(q_full, TILE_BYTES);
+    tma_load_2d(sQ, &tmQ, q_full, col0, q0);
+    tma_load_2d(sQ + HALF, &tmQ, q_full, col0 + 64, q0);
+    int nk_issued = 0, nv_issued = 0;
+    for (int j = 0; j < n_kv; ++j) {
+      const int st = j & 1;
+      const uint32_t par = ((j >> 1) & 1) ^ 1;
+      const int r0 = seg0 + j * TILE;
+      if (!mbar_wait(&k_empty[st], par, abort_flag, p.err)) break;
+      uint8_t* sK = smem + OFF_K + st * TILE_BYTES;
+      mbar_arrive_expect_tx(&k_full[st], TILE_BYTES);
+      tma_load_2d(sK, &tmK, &k_full[st], col0, r0);
+      tma_load_2d(sK + HALF, &tmK, &k_full[st], col0 + 64, r0);
+      ++nk_issued;
+      if (!mbar_wait(&v_empty[st], par, abort_flag, p.err)) break;
+      uint8_t* sV = smem + OFF_V + st * TILE_BYTES;
+      mbar_arrive_expect_tx(&v_full[st], TILE_BYTES);
+      tma_load_2d(sV, &tmV, &v_full[st], col0, r0);
+      tma_load_2d(sV + HALF, &tmV, &v_full[st], col0 + 64, r0);
+      ++nv_issued;
+    }
+    if (*abort_flag) {
+      int dummy = 0;
+      mbar_wait(q_full, 0, &dummy);
+      for (int j = (nk_issued > 2 ? nk_issued - 2 : 0); j < nk_issued; ++j)
+        mbar_wait(&k_full[j & 1], (j >> 1) & 1, &dummy);
+      for (int j = (nv_issued > 2 ? nv_issued - 2 : 0); j < nv_issued; ++j)
+        mbar_wait(&v_full[j & 1], (j >> 1) & 1, &dummy);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t id_s = idesc_bf16_f32(TILE, TILE);                // K-major A and B
+    const uint32_t id_o = idesc_bf16_f32(TILE, HD, false, true);     // B (V) MN-major
+    const uint32_t aQ = smem_u32(smem + OFF_Q);
+    const uint32_t aP = smem_u32(smem + OFF_P);
+    auto issue_pv = [&](int i) -> bool {
+      if (!mbar_wait(p_full, i & 1, abort_flag, p.err)) return false;
+      if (!mbar_wait(&v_full[i & 1], (i >> 1) & 1, abort_flag, p.err)) return false;
+      tc_fence_after();
+      const uint32_t aV = smem_u32(smem + OFF_V + (i & 1) * TILE_BYTES);
+#pragma unroll
+      for (int k = 0; k < TILE / 16; ++k) {
+        const uint64_t ad = sdesc_kmajor_sw128(aP + (k >> 2) * HALF + (k & 3) * 32);
+        const uint64_t bd = sdesc_mnmajor_sw128(aV + k * 16 * 128, HALF, 1024);
+        umma_bf16_ss(tmem + 256, ad, bd, id_o, (i | k) != 0 ? 1u : 0u);
+      }
+      umma_commit(&v_empty[i & 1]);
+      umma_commit(pv_done);
+      return true;
+    };
+    bool ok = mbar_wait(q_full, 0, abort_flag, p.err);
+    for (int j = 0; ok && j < n_kv; ++j) {
+      const int st = j & 1;
+      if (!mbar_wait(&s_empty[st], ((j >> 1) & 1) ^ 1, abort_flag, p.err)) { ok = false; break; }
+      if (!mbar_wait(&k_full[st], (j >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t aK = smem_u32(smem + OFF_K + st * TILE_BYTES);
+#pragma unroll
+      for (int k = 0; k < HD / 16; ++k) {
+        const uint32_t off = (k >> 2) * HALF + (k & 3) * 32;
+        umma_bf16_ss(tmem + st * TILE, sdesc_kmajor_sw128(aQ + off), sdesc_kmajor_sw128(aK + off), id_s,
+                     k != 0 ? 1u : 0u);
+      }
+      umma_commit(&k_empty[st]);
+      umma_commit(&s_full[st]);
+      if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+    }
+    if (ok) issue_pv(n_kv - 1);
+    umma_commit(mma_done);
+    int dummy = 0;
+    mbar_wait(mma_done, 0, &dummy);
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ softmax
+    const int lg = warp & 3;
+    const int row = lg * 32 + lane;  // query row inside the tile == TMEM lane
+    const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
+    uint8_t* sP = smem + OFF_P;
+    float m_ref = -INFINITY, l_sum = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kv; ++j) {
+      const int st = j & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[st], (j >> 1) & 1, abort_flag, p.err));
+      if (!ok) break;
+      tc_fence_after();
+      float s[TILE];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_off + st * TILE + c * 32, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(r[e]) * p.scale_log2;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_empty[st]);
+      const int valid = L - j * TILE;  // keys past the segment end are excluded
+      if (valid < TILE) {
+#pragma unroll
+        for (int e = 0; e < TILE; ++e)
+          if (e >= valid) s[e] = -INFINITY;
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < TILE; ++e) mx = fmaxf(mx, s[e]);
+      float alpha = 1.f;
+      bool move = false;
+      if (j == 0) {
+        m_ref = mx;
+      } else if (mx > m_ref + kRescaleThreshold) {
+        alpha = ex2(m_ref - mx);
+        m_ref = mx;
+        move = true;
+      }
+      l_sum *= alpha;
+      uint32_t pk[TILE / 2];
+      float part = 0.f;
+#pragma unroll
+      for (int e = 0; e < TILE / 2; ++e) {
+        const float p0 = ex2(s[2 * e] - m_ref);
+        const float p1 = ex2(s[2 * e + 1] - m_ref);
+        part += p0 + p1;
+        pk[e] = pack_bf16x2(p0, p1);
+      }
+      l_sum += part;
+      if (j >= 1) {  // P buffer free and O stable once PV of the previous tile is done
+        ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (j - 1) & 1, abort_flag, p.err));
+        if (!ok) break;
+        tc_fence_after();
+      }
+      if (__any_sync(0xffffffffu, move)) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_off + 256 + c * 32, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+          tmem_st32(tmem + lane_off + 256 + c * 32, r);
+        }
+        tmem_st_wait();
+      }
+      // P row -> smem, K-major with the 128-byte swizzle: 16-byte chunk ch of row r
+      // sits at r*128 + ((ch ^ (r & 7)) * 16) inside its 64-column half.
+#pragma unroll
+      for (int ch = 0; ch < 16; ++ch) {
+        const int half = ch >> 3, cw = ch & 7;
+        uint8_t* dst = sP + half * HALF + row * 128 + ((cw ^ (row & 7)) << 4);
+        *reinterpret_cast<uint4*>(dst) = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (n_kv - 1) & 1, abort_flag, p.err));
+    if (ok) {
+      tc_fence_after();
+      const int qrow = qt * TILE + row;
+      const float inv = 1.0f / l_sum;
+      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) + (size_t)(seg0 + qrow) * p.ldo + col0;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        __syncwarp();
+        tmem_ld32(tmem + lane_off + 256 + c * 32, r);
+        tmem_ld_wait();
+        if (qrow < L) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * e]) * inv, __uint_as_float(r[8 * e + 1]) * inv),
+                                pack_bf16x2(__uint_as_float(r[8 * e + 2]) * inv, __uint_as_float(r[8 * e + 3]) * inv),
+                                pack_bf16x2(__uint_as_float(r[8 * e + 4]) * inv, __uint_as_float(r[8 * e + 5]) * inv),
+                                pack_bf16x2(__uint_as_float(r[8 * e + 6]) * inv, __uint_as_float(r[8 * e + 7]) * inv));
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+zdit_status launch_attention(const AttnArgs& a, cudaStream_t s) {
+  if (a.T <= 0 || a.batch <= 0 || a.n_heads <= 0) return ZDIT_ERR_SHAPE;
+  if (a.ldq % 8 || a.ldk % 8 || a.ldv % 8 || a.ldo % 8) return ZDIT_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(a.q) | reinterpret_cast<uintptr_t>(a.k) | reinterpret_cast<uintptr_t>(a.v) |
+       reinterpret_cast<uintptr_t>(a.o)) & 15)
+    return ZDIT_ERR_ALIGNMENT;
+  int total_qt = 0;
+  for (int b = 0; b < a.batch; ++b) {
+    const int L = a.cu_seqlens_host[b + 1] - a.cu_seqlens_host[b];
+    if (L <= 0) return ZDIT_ERR_SHAPE;
+    total_qt += (L + TILE - 1) / TILE;
+  }
+  if (a.cu_seqlens_host[0] != 0 || a.cu_seqlens_host[a.batch] > a.T) return ZDIT_ERR_SHAPE;
+  CUtensorMap tq, tk, tv;
+  const int cols = a.n_heads * HD;
+  if (!make_tmap_bf16_2d(&tq, a.q, a.T, cols, a.ldq, TILE, 64)) return ZDIT_ERR_CUDA;
+  if (!make_tmap_bf16_2d(&tk, a.k, a.T, cols, a.ldk, TILE, 64)) return ZDIT_ERR_CUDA;
+  if (!make_tmap_bf16_2d(&tv, a.v, a.T, cols, a.ldv, TILE, 64)) return ZDIT_ERR_CUDA;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
+      return ZDIT_ERR_CUDA;
+    attr = true;
+  }
+  AParams p;
+  p.ldo = a.ldo;
+  p.n_heads = a.n_heads;
+  p.batch = a.batch;
+  p.o = a.o;
+  p.cu = a.cu_seqlens_dev;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  p.err = device_error_ptr();
+  dim3 grid(total_qt, a.n_heads);
+  attn_tc_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? ZDIT_OK : ZDIT_ERR_CUDA;
+}
+
+}  // namespace zdit

@@ -1,0 +1,389 @@
+// Persistent tcgen05 GEMM for sm_100a with fused epilogues.
+//
+//   C[M, N] = A[M, K] . B[N, K]^T,  A and B bf16 row-major (K contiguous), fp32 TMEM
+//   accumulator, 128 x 256 output tile per CTA, 64-deep K slices.
+//
+// Warp roles (192 threads, one CTA per SM):
+//   warp 0  lane 0 : TMA producer, 4-stage smem ring (A 16 KB + B 32 KB per stage)
+//   warp 1  lane 0 : tcgen05.mma issuer; warp 1 also owns the TMEM allocation
+//   warps 2-5      : epilogue; TMEM lane group (warp % 4) -> 32 output rows each
+// The accumulator is double-buffered in TMEM (2 x 256 columns) so the epilogue of
+// tile i overlaps the main loop of tile i + 1.
+//
+// Epilogues (the DiT block's projection steps, "Z-Image-Turbo port" DiT row and
+// "Native creative jobs", "Recipes and precision": FP32 accumulators, SwiGLU gate in
+// FP32, bf16 storage, never fp16):
+//   EPI_F32    fp32 store (+ bias)                 out-proj, w2, embedders
+//   EPI_BF16   bf16 store (+ bias)
+//   EPI_QKV    q/k columns: optional per-head RMSNorm, then real interleaved RoPE
+//              with per-token cos/sin; bf16 store of [q | k | v]
+//   EPI_SWIGLU gate/up column blocks -> silu(gate) * up, bf16 store
+#include <cudaTypedefs.h>
+
+#include <cstdio>
+#include <mutex>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace zdit {
+
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_TILE = BM * BK * 2;  // 16 KB
+constexpr int B_TILE = BN * BK * 2;  // 32 KB
+constexpr int STAGE_BYTES = A_TILE + B_TILE;
+constexpr int THREADS = 192;
+constexpr int TMEM_COLS = 2 * BN;
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+
+struct KParams {
+  int M, N, K, ldo;
+  void* out;
+  const float* bias;
+  const float* rcos;
+  const float* rsin;
+  const float* qn;
+  const float* kn;
+  float eps;
+  int dim;
+  int num_m, num_n, num_k, group_m;
+  int* err;
+};
+
+__device__ __forceinline__ void tile_coords(int t, const KParams& p, int& mb, int& nb) {
+  const int group = p.group_m * p.num_n;
+  const int g = t / group;
+  const int first = g * p.group_m;
+  const int gm = min(p.num_m - first, p.group_m);
+  const int r = t - g * group;
+  mb = first + r % gm;
+  nb = r / gm;
+}
+
+__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+
+template <int EPI>
+__device__ __forceinline__ void epilogue_tile(const KParams& p, uint32_t taddr, int row, int nb) {
+  const bool row_ok = row < p.M;
+  if constexpr (EPI == EPI_F32 || EPI == EPI_BF16) {
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      const int col0 = nb * BN + c * 32;
+      if (col0 >= p.N) break;  // warp-uniform
+      uint32_t r[32];
+      __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the row-masked stores
+      tmem_ld32(taddr + c * 32, r);
+      tmem_ld_wait();
+      float v[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+      if (p.bias != nullptr) {
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+          const float4 b = *reinterpret_cast<const float4*>(p.bias + col0 + j);
+          v[j] += b.x; v[j + 1] += b.y; v[j + 2] += b.z; v[j + 3] += b.w;
+        }
+      }
+      if (row_ok) {
+        if constexpr (EPI == EPI_F32) {
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + (size_t)row * p.ldo + col0);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.ldo + col0);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            dst[j] = make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
+                                pack_bf16x2(v[8 * j + 4], v[8 * j + 5]), pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+        }
+      }
+    }
+  } else if constexpr (EPI == EPI_SWIGLU) {
+    // tile columns [0,128) hold gate rows 128*nb.., [128,256) the matching up rows
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      uint32_t g[32], u[32];
+      __syncwarp();
+      tmem_ld32(taddr + c * 32, g);
+      tmem_ld32(taddr + 128 + c * 32, u);
+      tmem_ld_wait();
+      if (row_ok) {
+        uint32_t h[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float h0 = silu_f(__uint_as_float(g[2 * j])) * __uint_as_float(u[2 * j]);
+          const float h1 = silu_f(__uint_as_float(g[2 * j + 1])) * __uint_as_float(u[2 * j + 1]);
+          h[j] = pack_bf16x2(h0, h1);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.ldo +
+                                              nb * 128 + c * 32);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) dst[j] = make_uint4(h[4 * j], h[4 * j + 1], h[4 * j + 2], h[4 * j + 3]);
+      }
+    }
+  } else if constexpr (EPI == EPI_QKV) {
+#pragma unroll 1
+    for (int hh = 0; hh < BN / 128; ++hh) {
+      const int colh = nb * BN + hh * 128;
+      float v[128];
+      __syncwarp();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(taddr + hh * 128 + c * 32, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[c * 32 + j] = __uint_as_float(r[j]);
+      }
+      if (!row_ok) continue;
+      const bool is_q = colh < p.dim;
+      const bool is_k = !is_q && colh < 2 * p.dim;
+      if (is_q || is_k) {
+        const float* nw = is_q ? p.qn : p.kn;
+        if (nw != nullptr) {
+          float ss = 0.f;
+#pragma unroll
+          for (int j = 0; j < 128; ++j) ss += v[j] * v[j];
+          const float rinv = 1.0f / sqrtf(ss * (1.0f / 128.0f) + p.eps);
+#pragma unroll
+          for (int j = 0; j < 128; ++j) v[j] = v[j] * rinv * nw[j];
+        }
+        const float4* cs = reinterpret_cast<const float4*>(p.rcos + (size_t)row * 64);
+        const float4* sn = reinterpret_cast<const float4*>(p.rsin + (size_t)row * 64);
+#pragma unroll
+        for (int i4 = 0; i4 < 16; ++i4) {
+          const float4 c4 = cs[i4], s4 = sn[i4];
+          const float cc[4] = {c4.x, c4.y, c4.z, c4.w};
+          const float ssn[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = i4 * 4 + e;
+            const float x0 = v[2 * i], x1 = v[2 * i + 1];
+            v[2 * i] = x0 * cc[e] - x1 * ssn[e];
+            v[2 * i + 1] = x0 * ssn[e] + x1 * cc[e];
+          }
+        }
+      }
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.ldo + colh);
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        dst[j] = make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
+                            pack_bf16x2(v[8 * j + 4], v[8 * j + 5]), pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+    }
+  }
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(THREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const KParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* done = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 4);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int num_tiles = p.num_m * p.num_n;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ TMA producer
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t armed = 0;  // bit s: stage s has an armed phase; parity in armed_par
+    uint32_t armed_par = 0;
+    for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
+      int mb, nb;
+      tile_coords(t, p, mb, nb);
+      for (int kb = 0; kb < p.num_k; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err)) break;
+        uint8_t* sa = smem + stage * STAGE_BYTES;
+        mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+        tma_load_2d(sa, &tmA, &full[stage], kb * BK, mb * BM);
+        tma_load_2d(sa + A_TILE, &tmB, &full[stage], kb * BK, nb * BN);
+        armed |= 1u << stage;
+        armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    if (*abort_flag) {
+      // let copies already in flight land before the CTA's shared memory is released
+      int dummy = 0;
+      for (int s = 0; s < STAGES; ++s)
+        if (armed & (1u << s)) mbar_wait(&full[s], (armed_par >> s) & 1u, &dummy);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t idesc = idesc_bf16_f32(BM, BN);
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
+      if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.err)) break;
+      tc_fence_after();
+      const uint32_t d = tmem_base + acc * BN;
+      bool ok = true;
+      for (int kb = 0; kb < p.num_k; ++kb) {
+        if (!mbar_wait(&full[stage], phase, abort_flag, p.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(smem + stage * STAGE_BYTES);
+        const uint32_t b0 = a0 + A_TILE;
+#pragma unroll
+        for (int k = 0; k < BK / 16; ++k)
+          umma_bf16_ss(d, sdesc_kmajor_sw128(a0 + k * 32), sdesc_kmajor_sw128(b0 + k * 32), idesc,
+                       (kb | k) != 0 ? 1u : 0u);
+        umma_commit(&empty[stage]);
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (!ok) break;
+      umma_commit(&tfull[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1;
+    }
+    // all MMAs issued by this thread have finished once `done` fires
+    umma_commit(done);
+    int dummy = 0;
+    mbar_wait(done, 0, &dummy);
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ epilogue
+    const int lg = warp & 3;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err));
+      if (!ok) break;
+      tc_fence_after();
+      int mb, nb;
+      tile_coords(t, p, mb, nb);
+      const uint32_t taddr = tmem_base + ((uint32_t)(lg * 32) << 16) + acc * BN;
+      epilogue_tile<EPI>(p, taddr, mb * BM + lg * 32 + lane, nb);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1;
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+template <int EPI>
+zdit_status launch_epi(const CUtensorMap& ta, const CUtensorMap& tb, const KParams& kp, int grid,
+                       cudaStream_t s) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(gemm_tc_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
+        cudaSuccess)
+      return ZDIT_ERR_CUDA;
+    attr_set = true;
+  }
+  gemm_tc_kernel<EPI><<<grid, THREADS, SMEM_BYTES, s>>>(ta, tb, kp);
+  return cudaGetLastError() == cudaSuccess ? ZDIT_OK : ZDIT_ERR_CUDA;
+}
+
+}  // namespace
+
+bool make_tmap_bf16_2d(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint64_t ld_elems,
+                       uint32_t box_rows, uint32_t box_cols) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld_elems * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+zdit_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
+  if (a.M <= 0 || a.N <= 0 || a.K <= 0) return ZDIT_ERR_SHAPE;
+  if (a.K % 8 || a.lda % 8 || a.ldb % 8 || a.N % 32) return ZDIT_ERR_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(a.A) | reinterpret_cast<uintptr_t>(a.B) |
+       reinterpret_cast<uintptr_t>(a.out)) & 15)
+    return ZDIT_ERR_ALIGNMENT;
+  if (a.epi == EPI_SWIGLU && (a.N % BN)) return ZDIT_ERR_SHAPE;
+  if (a.epi == EPI_QKV && (a.N != 3 * a.dim || a.dim % 128 || a.N % BN || !a.rope_cos || !a.rope_sin))
+    return ZDIT_ERR_SHAPE;
+  if ((a.epi == EPI_F32 || a.epi == EPI_BF16) && (a.ldo % 4)) return ZDIT_ERR_ALIGNMENT;
+  CUtensorMap ta, tb;
+  if (!make_tmap_bf16_2d(&ta, a.A, a.M, a.K, a.lda, BM, BK)) return ZDIT_ERR_CUDA;
+  if (!make_tmap_bf16_2d(&tb, a.B, a.N, a.K, a.ldb, BN, BK)) return ZDIT_ERR_CUDA;
+  KParams kp;
+  kp.M = a.M; kp.N = a.N; kp.K = a.K; kp.ldo = a.ldo; kp.out = a.out; kp.bias = a.bias;
+  kp.rcos = a.rope_cos; kp.rsin = a.rope_sin; kp.qn = a.qn; kp.kn = a.kn; kp.eps = a.eps; kp.dim = a.dim;
+  kp.num_m = (a.M + BM - 1) / BM;
+  kp.num_n = (a.N + BN - 1) / BN;
+  kp.num_k = (a.K + BK - 1) / BK;
+  kp.group_m = 16;
+  kp.err = device_error_ptr();
+  const int tiles = kp.num_m * kp.num_n;
+  const int grid = tiles < num_sms() ? tiles : num_sms();
+  switch (a.epi) {
+    case EPI_F32: return launch_epi<EPI_F32>(ta, tb, kp, grid, s);
+    case EPI_BF16: return launch_epi<EPI_BF16>(ta, tb, kp, grid, s);
+    case EPI_QKV: return launch_epi<EPI_QKV>(ta, tb, kp, grid, s);
+    case EPI_SWIGLU: return launch_epi<EPI_SWIGLU>(ta, tb, kp, grid, s);
+  }
+  return ZDIT_ERR_INVALID_ARG;
+}
+
+}  // namespace zdit

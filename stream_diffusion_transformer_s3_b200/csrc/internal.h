@@ -1,0 +1,94 @@
+// Internal interfaces between the C-ABI layer and the kernel translation units.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "../../include/zdit.h"
+
+namespace zdit {
+
+// ---------------------------------------------------------------- GEMM (tcgen05)
+// C[M, N] = A[M, K] . B[N, K]^T with bf16 A, B (both K-major, row-major in memory)
+// and an fp32 accumulator in TMEM, followed by one of the fused epilogues.
+enum GemmEpilogue : int {
+  EPI_F32 = 0,     // out fp32 [M, ldo] = acc (+ bias[n])
+  EPI_BF16 = 1,    // out bf16 [M, ldo] = acc (+ bias[n])
+  EPI_QKV = 2,     // out bf16 [M, 3D]; columns < 2D: optional per-head RMSNorm, then RoPE
+  EPI_SWIGLU = 3,  // out bf16 [M, N/2]; tile columns [gate 128 | up 128] -> silu(g) * u
+};
+
+struct GemmArgs {
+  const void* A;  // bf16 [M, K], row stride lda elements
+  const void* B;  // bf16 [N, K], row stride ldb elements
+  int M, N, K, lda, ldb;
+  int epi;
+  void* out;
+  int ldo;
+  const float* bias;      // [N] or nullptr (EPI_F32 / EPI_BF16)
+  const float* rope_cos;  // [M, 64] (EPI_QKV)
+  const float* rope_sin;
+  int dim;                // D (EPI_QKV): columns < 2D are q | k
+  const float* qn;        // [128] per-head RMSNorm weights (EPI_QKV, optional)
+  const float* kn;
+  float eps;
+};
+
+zdit_status launch_gemm(const GemmArgs& a, cudaStream_t s);
+
+// ---------------------------------------------------------------- attention
+struct AttnArgs {
+  const void* q;  // bf16 [T, ldq] ; head h at columns h*128 .. h*128+127
+  const void* k;
+  const void* v;
+  int ldq, ldk, ldv;  // row strides in elements
+  void* o;            // bf16 [T, ldo]
+  int ldo;
+  int T, n_heads, batch;
+  const int* cu_seqlens_dev;   // [batch + 1]
+  const int* cu_seqlens_host;  // [batch + 1]
+  float scale;                 // 1 / sqrt(head_dim)
+};
+zdit_status launch_attention(const AttnArgs& a, cudaStream_t s);
+
+// ---------------------------------------------------------------- row / small kernels
+struct RowModArgs {
+  const float* x;        // [T, D]
+  int T, D;
+  const float* w;        // [D] norm weight
+  const float* mod;      // per-branch modulation base or nullptr; scale at mod[b*mod_stride + d]
+  int mod_stride;
+  const int* cu_seqlens; // [B + 1] device (branch of each row)
+  int batch;
+  float eps;
+  __nv_bfloat16* out;    // [T, D]
+};
+void launch_norm_modulate(const RowModArgs& a, cudaStream_t s);
+
+struct ResidArgs {
+  float* x;              // [T, D] in/out residual stream
+  const float* y;        // [T, D] projection output
+  int T, D;
+  const float* post_w;   // sandwich norm weight or nullptr (no post-norm)
+  const float* gate;     // per-branch gate: gate[b*gate_stride + d], or nullptr (gate 1)
+  int gate_stride;
+  int tanh_gate;
+  const int* cu_seqlens;
+  int batch;
+  float eps;
+  // optional fused next pre-norm: a = RMS(x_new) * w_next * (1 + scale_next[b])
+  const float* next_w;
+  const float* next_scale;
+  int next_scale_stride;
+  __nv_bfloat16* next_out;
+};
+void launch_residual(const ResidArgs& a, cudaStream_t s);
+
+
+int num_sms();
+
+// Device address of the library's latched device-error word on the current device.
+int* device_error_ptr();
+
+}  // namespace zdit

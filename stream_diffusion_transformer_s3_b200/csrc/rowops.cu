@@ -1,0 +1,504 @@
+// Bandwidth-bound row and element kernels of the DiT hot path.
+//
+//   norm_modulate : a = Norm(x) * w * (1 + scale_b) -> bf16 GEMM operand
+//                   (RMSNorm pre-norm of the block; LayerNorm without affine for the
+//                   final layer; plain RMSNorm for the caption embedder)
+//   residual      : x += gate_b * PostNorm(y), optionally fused with the next
+//                   pre-norm so x is read once per step
+//   adaln_gemv    : m_b = W_ada temb_b + b_ada (weight-streaming GEMV)
+//   euler_cfg     : x += (sigma_next - sigma_cur) * -(pos + g (pos - neg))
+//   rope_table    : per-token cos/sin of the 3-axis rotary angles
+//   timestep_embed, patchify / unpatchify, casts and row fills
+//
+// Row kernels use one 256-thread CTA per row; each thread keeps up to MAXV float4 of
+// the row in registers so the row is read from HBM exactly once.
+#include <cuda_bf16.h>
+
+#include <cmath>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace zdit {
+
+// Latched device-side error word (0 = none); kernels get its address as a
+// parameter; zdit_device_status reads and clears it.
+__device__ int g_device_error = 0;
+
+int* device_error_ptr() {
+  static int* ptrs[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return nullptr;
+  if (ptrs[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) == cudaSuccess) ptrs[dev] = static_cast<int*>(p);
+  }
+  return ptrs[dev];
+}
+
+zdit_status read_and_clear_device_error() {
+  int err = 0;
+  if (cudaMemcpyFromSymbol(&err, g_device_error, sizeof(int)) != cudaSuccess) return ZDIT_ERR_CUDA;
+  if (err != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return ZDIT_ERR_CUDA;
+  }
+  return static_cast<zdit_status>(err);
+}
+
+namespace {
+
+constexpr int RT = 256;  // threads per row CTA
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float block_sum(float v, float* sh) {
+  v = warp_sum(v);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  if (l == 0) sh[w] = v;
+  __syncthreads();
+  float r = 0.f;
+#pragma unroll
+  for (int i = 0; i < RT / 32; ++i) r += sh[i];
+  __syncthreads();
+  return r;
+}
+
+__device__ __forceinline__ int branch_of(const int* cu, int batch, int t) {
+  int b = 0;
+  while (b + 1 < batch && t >= cu[b + 1]) ++b;
+  return b;
+}
+
+__device__ __forceinline__ void store_bf16x4(__nv_bfloat16* dst, float a, float b, float c, float d) {
+  uint2 u = make_uint2(pack_bf16x2(a, b), pack_bf16x2(c, d));
+  *reinterpret_cast<uint2*>(dst) = u;
+}
+
+struct NormModParams {
+  const float* x;
+  int D;
+  const float* w;
+  const float* mod;
+  int mod_stride;
+  const int* cu;
+  int batch;
+  int fixed_branch;
+  int layer_norm;
+  float eps;
+  __nv_bfloat16* out;
+};
+
+template <int MAXV>
+__global__ void __launch_bounds__(RT) norm_modulate_kernel(NormModParams p) {
+  __shared__ float sh[RT / 32];
+  const int t = blockIdx.x;
+  const float* xr = p.x + (size_t)t * p.D;
+  float4 v[MAXV];
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int idx = (i * RT + threadIdx.x) * 4;
+    v[i] = idx < p.D ? *reinterpret_cast<const float4*>(xr + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  float mean = 0.f;
+  if (p.layer_norm) {
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) s += v[i].x + v[i].y + v[i].z + v[i].w;
+    mean = block_sum(s, sh) / p.D;
+  }
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int idx = (i * RT + threadIdx.x) * 4;
+    if (idx < p.D) {
+      const float a = v[i].x - mean, b = v[i].y - mean, c = v[i].z - mean, d = v[i].w - mean;
+      ss += a * a + b * b + c * c + d * d;
+    }
+  }
+  const float rstd = 1.0f / sqrtf(block_sum(ss, sh) / p.D + p.eps);
+  const int br = p.cu != nullptr ? branch_of(p.cu, p.batch, t) : p.fixed_branch;
+  const float* sc = p.mod != nullptr ? p.mod + (size_t)br * p.mod_stride : nullptr;
+  __nv_bfloat16* orow = p.out + (size_t)t * p.D;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int idx = (i * RT + threadIdx.x) * 4;
+    if (idx < p.D) {
+      float4 w4 = p.w != nullptr ? *reinterpret_cast<const float4*>(p.w + idx) : make_float4(1.f, 1.f, 1.f, 1.f);
+      if (sc != nullptr) {
+        const float4 s4 = *reinterpret_cast<const float4*>(sc + idx);
+        w4.x *= 1.f + s4.x; w4.y *= 1.f + s4.y; w4.z *= 1.f + s4.z; w4.w *= 1.f + s4.w;
+      }
+      store_bf16x4(orow + idx, (v[i].x - mean) * rstd * w4.x, (v[i].y - mean) * rstd * w4.y,
+                   (v[i].z - mean) * rstd * w4.z, (v[i].w - mean) * rstd * w4.w);
+    }
+  }
+}
+
+struct ResidParams {
+  float* x;
+  const float* y;
+  int D;
+  const float* post_w;
+  const float* gate;
+  int gate_stride;
+  int tanh_gate;
+  const int* cu;
+  int batch;
+  float eps;
+  const float* next_w;
+  const float* next_scale;
+  int next_scale_stride;
+  __nv_bfloat16* next_out;
+};
+
+template <int MAXV>
+__global__ void __launch_bounds__(RT) residual_kernel(ResidParams p) {
+  __shared__ float sh[RT / 32];
+  const int t = blockIdx.x;
+  const float* yr = p.y + (size_t)t * p.D;
+  float* xr = p.x + (size_t)t * p.D;
+  float4 y[MAXV];
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int idx = (i * RT + threadIdx.x) * 4;
+    y[i] = idx < p.D ? *reinterpret_cast<const float4*>(yr + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
+    ss += y[i].x * y[i].x + y[i].y * y[i].y + y[i].z * y[i].z + y[i].w * y[i].w;
+  }
+  float r = 1.f;
+  if (p.post_w != nullptr) r = 1.0f / sqrtf(block_sum(ss, sh) / p.D + p.eps);
+  const int br = branch_of(p.cu, p.batch, t);
+  const float* g = p.gate != nullptr ? p.gate + (size_t)br * p.gate_stride : nullptr;
+  float ss2 = 0.f;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int idx = (i * RT + threadIdx.x) * 4;
+    if (idx < p.D) {
+      float4 x4 = *reinterpret_cast<const float4*>(xr + idx);
+      float4 w4 = p.post_w != nullptr ? *reinterpret_cast<const float4*>(p.post_w + idx)
+                                      : make_float4(1.f, 1.f, 1.f, 1.f);
+      float4 g4 = g != nullptr ? *reinterpret_cast<const float4*>(g + idx) : make_float4(1.f, 1.f, 1.f, 1.f);
+      if (p.tanh_gate && g != nullptr) {
+        g4.x = tanhf(g4.x); g4.y = tanhf(g4.y); g4.z = tanhf(g4.z); g4.w = tanhf(g4.w);
+      }
+      x4.x += g4.x * (y[i].x * r * w4.x);
+      x4.y += g4.y * (y[i].y * r * w4.y);
+      x4.z += g4.z * (y[i].z * r * w4.z);
+      x4.w += g4.w * (y[i].w * r * w4.w);
+      *reinterpret_cast<float4*>(xr + idx) = x4;
+      y[i] = x4;  // keep the updated residual for the fused next norm
+      ss2 += x4.x * x4.x + x4.y * x4.y + x4.z * x4.z + x4.w * x4.w;
+    }
+  }
+  if (p.next_out == nullptr) return;  // uniform across the CTA
+  const float r2 = 1.0f / sqrtf(block_sum(ss2, sh) / p.D + p.eps);
+  const float* sc = p.next_scale != nullptr ? p.next_scale + (size_t)br * p.next_scale_stride : nullptr;
+  __nv_bfloat16* orow = p.next_out + (size_t)t * p.D;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int idx = (i * RT + threadIdx.x) * 4;
+    if (idx < p.D) {
+      float4 w4 = *reinterpret_cast<const float4*>(p.next_w + idx);
+      if (sc != nullptr) {
+        const float4 s4 = *reinterpret_cast<const float4*>(sc + idx);
+        w4.x *= 1.f + s4.x; w4.y *= 1.f + s4.y; w4.z *= 1.f + s4.z; w4.w *= 1.f + s4.w;
+      }
+      store_bf16x4(orow + idx, y[i].x * r2 * w4.x, y[i].y * r2 * w4.y, y[i].z * r2 * w4.z, y[i].w * r2 * w4.w);
+    }
+  }
+}
+
+// out[b * rows + r] = sum_e W[r, e] * temb[b, e] + bias[r]; one warp per row r,
+// 16-byte weight loads, temb staged in shared memory.
+__global__ void __launch_bounds__(256) adaln_gemv_kernel(const __nv_bfloat16* __restrict__ W,
+                                                         const float* __restrict__ bias,
+                                                         const float* __restrict__ temb, int B, int E, int rows,
+                                                         float* __restrict__ out) {
+  extern __shared__ float st[];  // [B, E]
+  for (int i = threadIdx.x; i < B * E; i += blockDim.x) st[i] = temb[i];
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.x * 8 + warp;
+  if (r >= rows) return;
+  float acc[8];
+#pragma unroll
+  for (int b = 0; b < 8; ++b) acc[b] = 0.f;
+  const __nv_bfloat16* wr = W + (size_t)r * E;
+  for (int e0 = lane * 8; e0 < E; e0 += 256) {
+    const uint4 u = *reinterpret_cast<const uint4*>(wr + e0);
+    const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&u);
+    float w[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) w[j] = __bfloat162float(h[j]);
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+      if (b < B) {
+        const float* tb = st + b * E + e0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[b] += w[j] * tb[j];
+      }
+    }
+  }
+#pragma unroll
+  for (int b = 0; b < 8; ++b) {
+    if (b < B) {
+      const float s = warp_sum(acc[b]);
+      if (lane == 0) out[(size_t)b * rows + r] = s + (bias != nullptr ? bias[r] : 0.f);
+    }
+  }
+}
+
+__global__ void euler_cfg_kernel(float* __restrict__ x, const float* __restrict__ vp,
+                                 const float* __restrict__ vn, int64_t n, float g, float dsig) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t n4 = n / 4;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride) {
+    float4 xv = reinterpret_cast<float4*>(x)[i];
+    const float4 p = reinterpret_cast<const float4*>(vp)[i];
+    float4 q = p;
+    if (vn != nullptr) q = reinterpret_cast<const float4*>(vn)[i];
+    // v = -(pos + g (pos - neg)); x += dsig * v
+    xv.x += dsig * -(p.x + g * (p.x - q.x));
+    xv.y += dsig * -(p.y + g * (p.y - q.y));
+    xv.z += dsig * -(p.z + g * (p.z - q.z));
+    xv.w += dsig * -(p.w + g * (p.w - q.w));
+    reinterpret_cast<float4*>(x)[i] = xv;
+  }
+  for (int64_t i = n4 * 4 + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+    const float p = vp[i];
+    const float q = vn != nullptr ? vn[i] : p;
+    x[i] += dsig * -(p + g * (p - q));
+  }
+}
+
+__global__ void rope_table_kernel(const int* __restrict__ pos, int64_t T, int half_dim, int a0, int a1, int a2,
+                                  double theta, float* __restrict__ cs, float* __restrict__ sn) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= T * half_dim) return;
+  const int64_t t = idx / half_dim;
+  const int i = (int)(idx % half_dim);
+  int axis, j, width;
+  if (i < a0 / 2) {
+    axis = 0; j = i; width = a0;
+  } else if (i < (a0 + a1) / 2) {
+    axis = 1; j = i - a0 / 2; width = a1;
+  } else {
+    axis = 2; j = i - (a0 + a1) / 2; width = a2;
+  }
+  const double omega = pow(theta, -2.0 * j / width);
+  const double phi = (double)pos[t * 3 + axis] * omega;
+  cs[idx] = (float)cos(phi);
+  sn[idx] = (float)sin(phi);
+}
+
+struct TembParams {
+  float t[8];
+};
+
+// temb_b = W2 . SiLU(W1 . [cos | sin](t_scale * t_b * freqs) + b1) + b2, E <= 1024.
+__global__ void timestep_embed_kernel(TembParams tp, int E, float t_scale, const __nv_bfloat16* __restrict__ w1,
+                                      const float* __restrict__ b1, const __nv_bfloat16* __restrict__ w2,
+                                      const float* __restrict__ b2, float* __restrict__ temb) {
+  extern __shared__ float sm[];  // [2E]
+  float* emb = sm;
+  float* hid = sm + E;
+  const int b = blockIdx.x;
+  const int half = E / 2;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int i = e % half;
+    const double freq = exp(-log(10000.0) * (double)i / (double)half);
+    const double arg = (double)t_scale * (double)tp.t[b] * freq;
+    emb[e] = (float)(e < half ? cos(arg) : sin(arg));
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    float a = b1[e];
+    for (int k = 0; k < E; ++k) a += __bfloat162float(w1[(size_t)e * E + k]) * emb[k];
+    hid[e] = a / (1.0f + expf(-a));
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    float a = b2[e];
+    for (int k = 0; k < E; ++k) a += __bfloat162float(w2[(size_t)e * E + k]) * hid[k];
+    temb[(size_t)b * E + e] = a;
+  }
+}
+
+// tokens[n, f] <-> latent[c, 2 hi + dy, 2 wi + dx] with n = hi * w + wi and
+// f = (dy * 2 + dx) * C + c; `dir` 0 = patchify, 1 = unpatchify.
+__global__ void patchify_kernel(const float* __restrict__ src, float* __restrict__ dst, int C, int h, int w,
+                                int dir) {
+  const int64_t total = (int64_t)h * w * 4 * C;
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= total) return;
+  const int F = 4 * C;
+  const int64_t n = idx / F;
+  const int f = (int)(idx % F);
+  const int q = f / C, c = f % C;
+  const int dy = q >> 1, dx = q & 1;
+  const int hi = (int)(n / w), wi = (int)(n % w);
+  const int64_t li = ((int64_t)c * (2 * h) + (2 * hi + dy)) * (2 * w) + (2 * wi + dx);
+  if (dir == 0)
+    dst[idx] = src[li];
+  else
+    dst[li] = src[idx];
+}
+
+__global__ void cast_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst, int64_t n) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) dst[i] = __float2bfloat16_rn(src[i]);
+}
+
+__global__ void fill_rows_kernel(float* __restrict__ x, int D, int nrows, const float* __restrict__ vec) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < (int64_t)nrows * D) x[i] = vec[i % D];
+}
+
+struct LayoutParams {
+  int B, grid_h, grid_w;
+  int n_cap[8];
+};
+
+// Token layout of the stack: branch b is [image (n_img) | caption (n_cap_b)].
+// Positions: image cell (h, w) -> (n_cap_b + 1, h, w); caption k -> (k + 1, 0, 0).
+// Writes the positions of the image-only, caption-only and joint sequences and the
+// three cu_seqlens arrays.
+__global__ void stack_layout_kernel(LayoutParams lp, int* __restrict__ pos_img, int* __restrict__ pos_cap,
+                                    int* __restrict__ pos_joint, int* __restrict__ cu_img, int* __restrict__ cu_cap,
+                                    int* __restrict__ cu_joint) {
+  const int n_img = lp.grid_h * lp.grid_w;
+  int joff[9], coff[9];
+  joff[0] = coff[0] = 0;
+  for (int b = 0; b < lp.B; ++b) {
+    joff[b + 1] = joff[b] + n_img + lp.n_cap[b];
+    coff[b + 1] = coff[b] + lp.n_cap[b];
+  }
+  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t == 0) {
+    for (int b = 0; b <= lp.B; ++b) {
+      cu_img[b] = b * n_img;
+      cu_cap[b] = coff[b];
+      cu_joint[b] = joff[b];
+    }
+  }
+  if (t >= joff[lp.B]) return;
+  int b = 0;
+  while (t >= joff[b + 1]) ++b;
+  const int local = (int)(t - joff[b]);
+  int p0, p1, p2;
+  if (local < n_img) {
+    p0 = lp.n_cap[b] + 1;
+    p1 = local / lp.grid_w;
+    p2 = local % lp.grid_w;
+    const int64_t ii = (int64_t)b * n_img + local;
+    pos_img[ii * 3] = p0; pos_img[ii * 3 + 1] = p1; pos_img[ii * 3 + 2] = p2;
+  } else {
+    const int k = local - n_img;
+    p0 = k + 1; p1 = 0; p2 = 0;
+    const int64_t ci = coff[b] + k;
+    pos_cap[ci * 3] = p0; pos_cap[ci * 3 + 1] = p1; pos_cap[ci * 3 + 2] = p2;
+  }
+  pos_joint[t * 3] = p0; pos_joint[t * 3 + 1] = p1; pos_joint[t * 3 + 2] = p2;
+}
+
+}  // namespace
+
+void launch_stack_layout(const int* n_cap, int B, int grid_h, int grid_w, int* pos_img, int* pos_cap, int* pos_joint,
+                         int* cu_img, int* cu_cap, int* cu_joint, cudaStream_t s) {
+  LayoutParams lp;
+  lp.B = B; lp.grid_h = grid_h; lp.grid_w = grid_w;
+  int64_t T = 0;
+  for (int b = 0; b < 8; ++b) {
+    lp.n_cap[b] = b < B ? n_cap[b] : 0;
+    if (b < B) T += (int64_t)grid_h * grid_w + n_cap[b];
+  }
+  stack_layout_kernel<<<(unsigned)((T + 255) / 256), 256, 0, s>>>(lp, pos_img, pos_cap, pos_joint, cu_img, cu_cap,
+                                                                  cu_joint);
+}
+
+void launch_norm_modulate_ex(const float* x, int T, int D, const float* w, const float* mod, int mod_stride,
+                             const int* cu, int batch, int fixed_branch, int layer_norm, float eps,
+                             __nv_bfloat16* out, cudaStream_t s) {
+  NormModParams p{x, D, w, mod, mod_stride, cu, batch, fixed_branch, layer_norm, eps, out};
+  const int v = (D + RT * 4 - 1) / (RT * 4);
+  if (T <= 0) return;
+  if (v <= 1)
+    norm_modulate_kernel<1><<<T, RT, 0, s>>>(p);
+  else if (v <= 2)
+    norm_modulate_kernel<2><<<T, RT, 0, s>>>(p);
+  else if (v <= 4)
+    norm_modulate_kernel<4><<<T, RT, 0, s>>>(p);
+  else
+    norm_modulate_kernel<8><<<T, RT, 0, s>>>(p);
+}
+
+void launch_norm_modulate(const RowModArgs& a, cudaStream_t s) {
+  launch_norm_modulate_ex(a.x, a.T, a.D, a.w, a.mod, a.mod_stride, a.cu_seqlens, a.batch, 0, 0, a.eps, a.out, s);
+}
+
+void launch_residual(const ResidArgs& a, cudaStream_t s) {
+  ResidParams p{a.x,       a.y,    a.D,          a.post_w,  a.gate,       a.gate_stride, a.tanh_gate,
+                a.cu_seqlens, a.batch, a.eps,    a.next_w,  a.next_scale, a.next_scale_stride, a.next_out};
+  const int v = (a.D + RT * 4 - 1) / (RT * 4);
+  if (a.T <= 0) return;
+  if (v <= 1)
+    residual_kernel<1><<<a.T, RT, 0, s>>>(p);
+  else if (v <= 2)
+    residual_kernel<2><<<a.T, RT, 0, s>>>(p);
+  else if (v <= 4)
+    residual_kernel<4><<<a.T, RT, 0, s>>>(p);
+  else
+    residual_kernel<8><<<a.T, RT, 0, s>>>(p);
+}
+
+void launch_gemv(const __nv_bfloat16* W, const float* bias, const float* temb, int B, int E, int rows, float* out,
+                 cudaStream_t s) {
+  adaln_gemv_kernel<<<(rows + 7) / 8, 256, (size_t)B * E * sizeof(float), s>>>(W, bias, temb, B, E, rows, out);
+}
+
+void launch_euler_cfg(float* x, const float* vp, const float* vn, int64_t n, float g, float dsig, cudaStream_t s) {
+  int blocks = (int)((n / 4 + 255) / 256);
+  if (blocks < 1) blocks = 1;
+  if (blocks > 4 * num_sms()) blocks = 4 * num_sms();
+  euler_cfg_kernel<<<blocks, 256, 0, s>>>(x, vp, vn, n, g, dsig);
+}
+
+void launch_rope_table(const int* pos, int64_t T, int head_dim, const int* axes, float theta, float* cs, float* sn,
+                       cudaStream_t s) {
+  const int64_t n = T * (head_dim / 2);
+  if (n <= 0) return;
+  rope_table_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(pos, T, head_dim / 2, axes[0], axes[1], axes[2],
+                                                                 (double)theta, cs, sn);
+}
+
+void launch_timestep_embed(const float* t_host, int B, int E, float t_scale, const __nv_bfloat16* w1,
+                           const float* b1, const __nv_bfloat16* w2, const float* b2, float* temb, cudaStream_t s) {
+  TembParams tp;
+  for (int i = 0; i < 8; ++i) tp.t[i] = i < B ? t_host[i] : 0.f;
+  timestep_embed_kernel<<<B, 256, 2 * E * sizeof(float), s>>>(tp, E, t_scale, w1, b1, w2, b2, temb);
+}
+
+void launch_patchify(const float* src, float* dst, int C, int h, int w, int dir, cudaStream_t s) {
+  const int64_t total = (int64_t)h * w * 4 * C;
+  if (total <= 0) return;
+  patchify_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(src, dst, C, h, w, dir);
+}
+
+void launch_cast_bf16(const float* src, __nv_bfloat16* dst, int64_t n, cudaStream_t s) {
+  if (n <= 0) return;
+  cast_bf16_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(src, dst, n);
+}
+
+void launch_fill_rows(float* x, int D, int nrows, const float* vec, cudaStream_t s) {
+  const int64_t n = (int64_t)nrows * D;
+  if (n <= 0) return;
+  fill_rows_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(x, D, nrows, vec);
+}
+
+}  // namespace zdit

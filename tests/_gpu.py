@@ -1,0 +1,64 @@
+"""Shared helpers of the GPU parity tests (device marshalling and error metrics)."""
+import numpy as np
+import pytest
+import torch
+
+import stream_diffusion_transformer_s3_b200 as Z
+
+
+def require_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    Z.lib()  # raises if the library is missing: no fallback
+
+
+def dev(a, dtype=torch.float32):
+    return torch.as_tensor(np.ascontiguousarray(a)).to(device="cuda", dtype=dtype).contiguous()
+
+
+def bf16(a):
+    return dev(np.asarray(a, np.float32), torch.bfloat16)
+
+
+def host(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def errors(got, ref):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    diff = np.abs(got - ref)
+    return {"rel_l2": float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300)),
+            "mean_abs": float(diff.mean()), "median_abs": float(np.median(diff)),
+            "max_abs": float(diff.max())}
+
+
+def rope_tables(pos, dims, stream=None):
+    T = pos.shape[0]
+    p = dev(pos.astype(np.int32), torch.int32)
+    cs = torch.empty(T, dims.head_dim // 2, device="cuda")
+    sn = torch.empty_like(cs)
+    Z.zdit_rope_table(p, dims.rope_axes, dims.rope_theta, cs, sn, dims.head_dim)
+    return cs, sn
+
+
+def dims_of(d):
+    return Z.Dims(dim=d.dim, n_heads=d.n_heads, head_dim=d.head_dim, ffn_hidden=d.ffn_hidden,
+                  temb_dim=d.temb_dim, rope_axes=d.rope_axes, norm_eps=d.norm_eps,
+                  rope_theta=d.rope_theta)
+
+
+def run_block_gpu(case, d, flags):
+    """Runs zdit_block_forward on a synth block case; returns the output rows."""
+    dims = dims_of(d)
+    fl = Z.flags_of(flags.adaln, flags.sandwich, flags.qk_norm, flags.tanh_gate)
+    w = Z.DeviceBlock(case["weights"])
+    vl = Z.DeviceVarlen(case["cu_seqlens"])
+    x = dev(case["x"])
+    temb = dev(case["temb"])
+    cs, sn = rope_tables(case["pos"], dims)
+    nbytes = Z.block_workspace_bytes(dims, fl, vl.total, len(case["cu_seqlens"]) - 1)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    Z.zdit_block_forward(dims, fl, w, vl, x, temb, cs, sn, ws)
+    assert Z.zdit_device_status() == 0
+    return host(x)

@@ -1,0 +1,126 @@
+"""CPU checks of the C-ABI library: it loads, exports every symbol the header
+declares, and its host-side logic (validation, workspace sizing, the sigma schedule)
+behaves as documented.  No call here reaches a GPU."""
+import ctypes as C
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle as O
+import stream_diffusion_transformer_s3_b200 as Z
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "zdit.h")
+
+
+def declared_symbols():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"ZDIT_API\s+[\w\s\*]+?\b(zdit_\w+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = Z.lib()
+    names = declared_symbols()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(Z._SIGS), "binding and header disagree"
+
+
+def test_version_and_status_strings():
+    L = Z.lib()
+    assert L.zdit_version() == 100
+    for code, name in Z.STATUS.items():
+        assert L.zdit_status_string(code).decode() == name
+
+
+def test_sigma_schedule_host_matches_oracle():
+    for n in (1, 8, 50):
+        got = np.array(Z.zdit_sigma_schedule(n), dtype=np.float64)
+        np.testing.assert_allclose(got, O.sigma_schedule(n), rtol=1e-7, atol=1e-8)
+        assert got[-1] == 0.0 and got[0] == 1.0
+    assert Z.lib().zdit_sigma_schedule(0, (C.c_float * 2)()) == -1
+
+
+def test_block_workspace_sizing():
+    d = Z.Dims()
+    f = Z.flags_of()
+    small = Z.block_workspace_bytes(d, f, 608, 2)
+    big = Z.block_workspace_bytes(d, f, 8352, 2)
+    assert 0 < small < big
+    # activations alone: a, o (bf16 D) + qkv/h (bf16 max(3D, F)) + y (fp32 D) per token
+    per_tok = 2 * 3840 * 2 + 2 * 11520 + 4 * 3840
+    assert big >= 8352 * per_tok
+    assert Z.block_workspace_bytes(Z.Dims(head_dim=64), f, 608, 2) == 0
+    assert Z.block_workspace_bytes(d, f, 0, 2) == 0
+    assert Z.block_workspace_bytes(d, f, 608, 9) == 0
+
+
+def _fake(n=1 << 20):
+    return C.c_void_p(n)
+
+
+def test_block_forward_rejects_bad_arguments_before_launch():
+    L = Z.lib()
+    d = Z.Dims(dim=256, n_heads=2, ffn_hidden=768)
+    cfg = d.cfg(Z.flags_of())
+    w = Z.BlockWeights(**{f: _fake() for f, _ in Z.BlockWeights._fields_})
+    cu = (C.c_int32 * 2)(0, 96)
+    vl = Z.Varlen(1, _fake(), cu)
+    args = lambda **k: dict(dict(cfg=C.byref(cfg), w=C.byref(w), vl=C.byref(vl), x=_fake(), temb=_fake(),
+                                 rc=_fake(), rs=_fake(), ws=_fake(1 << 20), wsb=1 << 40), **k)
+    call = lambda a: L.zdit_block_forward(a["cfg"], a["w"], a["vl"], a["x"], a["temb"], a["rc"], a["rs"],
+                                          a["ws"], a["wsb"], None)
+    assert call(args(x=None)) == -1
+    bad = d.cfg(Z.flags_of())
+    bad.head_dim = 64
+    assert call(args(cfg=C.byref(bad))) == -2
+    bad2 = d.cfg(Z.flags_of())
+    bad2.rope_axes[0] = 30
+    assert call(args(cfg=C.byref(bad2))) == -2
+    cu_bad = (C.c_int32 * 3)(0, 50, 40)
+    vl_bad = Z.Varlen(2, _fake(), cu_bad)
+    assert call(args(vl=C.byref(vl_bad))) == -2
+    w_nul = Z.BlockWeights(**{f: _fake() for f, _ in Z.BlockWeights._fields_})
+    w_nul.w_ada = None
+    assert call(args(w=C.byref(w_nul))) == -1
+    assert call(args(x=_fake((1 << 20) + 4))) == -3
+    assert call(args(ws=_fake((1 << 20) + 64))) == -3
+
+
+def test_stack_dims_validation():
+    d = Z.Dims(dim=256, n_heads=2, ffn_hidden=768)
+    cfg = Z.StackCfg(d.cfg(Z.flags_of()), 2, 2, 2, 64, 2560, 1000.0, 1e-6)
+    n_cap = (C.c_int32 * 2)(64, 32)
+    n_val = (C.c_int32 * 2)(45, 1)
+    t = (C.c_float * 2)(0.5, 0.5)
+    ok = Z.StackInputs(2, 8, 8, n_cap, n_val, _fake(), _fake(), t)
+    L = Z.lib()
+    assert L.zdit_stack_workspace_bytes(C.byref(cfg), C.byref(ok)) > 0
+    n_cap_bad = (C.c_int32 * 2)(60, 32)   # caption length not a multiple of 32
+    bad = Z.StackInputs(2, 8, 8, n_cap_bad, n_val, _fake(), _fake(), t)
+    assert L.zdit_stack_workspace_bytes(C.byref(cfg), C.byref(bad)) == 0
+    n_val_bad = (C.c_int32 * 2)(65, 1)    # more valid rows than caption slots
+    bad = Z.StackInputs(2, 8, 8, n_cap, n_val_bad, _fake(), _fake(), t)
+    assert L.zdit_stack_workspace_bytes(C.byref(cfg), C.byref(bad)) == 0
+    odd_grid = Z.StackInputs(2, 5, 5, n_cap, n_val, _fake(), _fake(), t)   # 25 image tokens
+    assert L.zdit_stack_workspace_bytes(C.byref(cfg), C.byref(odd_grid)) == 0
+
+
+def test_euler_rejects_null_and_misaligned():
+    L = Z.lib()
+    assert L.zdit_euler_cfg_step(None, _fake(), None, 16, 1.0, 1.0, 0.9, None) == -1
+    assert L.zdit_euler_cfg_step(_fake((1 << 20) + 4), _fake(), None, 16, 1.0, 1.0, 0.9, None) == -3
+    assert L.zdit_euler_cfg_step(_fake(), _fake(), None, 0, 1.0, 1.0, 0.9, None) == 0
+
+
+def test_gate_up_interleave_layout():
+    w1 = np.arange(256 * 3).reshape(256, 3)
+    w3 = -np.arange(256 * 3).reshape(256, 3)
+    g = Z.interleave_gate_up(w1, w3)
+    assert g.shape == (512, 3)
+    np.testing.assert_array_equal(g[0:128], w1[0:128])
+    np.testing.assert_array_equal(g[128:256], w3[0:128])
+    np.testing.assert_array_equal(g[256:384], w1[128:256])
+    np.testing.assert_array_equal(g[384:512], w3[128:256])

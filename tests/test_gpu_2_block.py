@@ -1,0 +1,61 @@
+"""Block-level parity on the GPU: zdit_block_forward against the oracle's
+block_forward on the tiny single-block case and the full-width cond/uncond pair.
+
+Tolerance: relative L2 error <= 2e-2 on the block output and, more strictly, on
+the block's update (output minus input); mean and median absolute errors are
+reported alongside."""
+import numpy as np
+import pytest
+
+import oracle as O
+from stream_diffusion_transformer_s3_b200 import synth
+from _gpu import errors, require_gpu, run_block_gpu
+
+pytestmark = pytest.mark.gpu
+TOL = 2e-2
+
+
+@pytest.fixture(autouse=True)
+def _gpu():
+    require_gpu()
+
+
+def _check(case, d, flags):
+    got = run_block_gpu(case, d, flags)
+    ref = O.block_forward(case["x"], case["cu_seqlens"], case["pos"], case["temb"], case["weights"], d, flags)
+    x0 = case["x"].astype(np.float64)
+    e_out = errors(got, ref)
+    e_upd = errors(got - x0, ref - x0)
+    print(f"\n{flags}: out {e_out}\n  update {e_upd}")
+    assert np.all(np.isfinite(got))
+    assert e_out["rel_l2"] <= TOL, e_out
+    assert e_upd["rel_l2"] <= TOL, e_upd
+    return e_upd
+
+
+@pytest.mark.parametrize("flags", [
+    O.Flags(),
+    O.Flags(sandwich=False),
+    O.Flags(qk_norm=True),
+    O.Flags(tanh_gate=True),
+    O.Flags(adaln=False),
+])
+def test_config1_block(flags):
+    case = synth.block_case(0, synth.TINY, 8, 8, [32], [25], adaln=flags.adaln, qk_norm=flags.qk_norm)
+    _check(case, synth.TINY, flags)
+
+
+def test_config1_two_branches_ragged():
+    # two branches of different caption length; segments not multiples of 128
+    case = synth.block_case(4, synth.TINY, 8, 8, [64, 32], [45, 1])
+    _check(case, synth.TINY, O.Flags())
+
+
+def test_config2_full_width_block():
+    case = synth.config2(0)
+    _check(case, synth.FULL, O.Flags())
+
+
+def test_config2_full_width_block_qk_norm_no_sandwich():
+    case = synth.block_case(1, synth.FULL, 16, 16, [64, 32], [45, 1], x_max=6.7e3, qk_norm=True)
+    _check(case, synth.FULL, O.Flags(sandwich=False, qk_norm=True))
