@@ -1,0 +1,400 @@
+#!/usr/bin/env python
+"""Benchmark of the Z-Image-Turbo single-stream DiT hot path on B200.
+
+One step = one sampler step of the 1024x1024 workload: the 34-block DiT forward
+(2 noise-refiner + 2 context-refiner + 30 main blocks + final layer) over the
+cond/uncond pair (4096 image tokens each, captions padded to 128 and 32 tokens)
+through zdit_stack_forward, then the fused negated-CFG FlowMatchEuler update
+through zdit_euler_cfg_step.  Metric: DiT forward TFLOP/s (algorithmic FLOPs of the
+forward / device time), with ms per step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (launched by torch.distributed.run) every rank runs an independent
+replica (the DiT forward has no data-path exchange on one image; images are
+independent), timings are the max over ranks, and `value` is the whole-job rate.
+`--impl reference` times the CPU float64 oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+D, H, HD, F, E = 3840, 30, 128, 10240, 256
+PATCH, CAP = 64, 2560
+GRID = (64, 64)
+N_CAPS, N_VALIDS = (128, 32), (100, 1)
+KINDS = ["noise"] * 2 + ["context"] * 2 + ["main"] * 30
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+WORKLOAD = ("1024x1024 DiT forward, 34 blocks (2 noise-refiner + 2 context-refiner + 30 main + final), "
+            "cond/uncond pair: 4096 image tokens each + captions 128 (100 valid) / 32 (1 valid), "
+            "width 3840, 30x128 heads, SwiGLU 10240, then fused negated-CFG Euler update (g=1)")
+
+
+def forward_flops() -> float:
+    """Algorithmic FLOPs of one DiT forward of the benchmark workload."""
+    n_img = GRID[0] * GRID[1]
+
+    def block(lengths):
+        T = sum(lengths)
+        return 2.0 * T * D * (3 * D + D + 3 * F) + sum(4.0 * D * L * L for L in lengths)
+
+    f = 2 * block([n_img] * 2) + 2 * block(list(N_CAPS)) + 30 * block([n_img + c for c in N_CAPS])
+    f += 2.0 * 2 * n_img * PATCH * D + 2.0 * sum(N_VALIDS) * CAP * D + 2.0 * 2 * n_img * D * PATCH
+    f += 32 * 2.0 * 2 * E * 4 * D + 2.0 * 2 * E * D
+    return f
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            return json.load(fh), "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+# ------------------------------------------------------------------ clocks sampling
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.path = os.path.join("/tmp", f"zdit_clocks_{os.getpid()}.csv")
+        self.proc = None
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", gpu_id, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ our arm
+BLOCK_WORKLOAD = ("one main DiT block of the 1024x1024 workload: joint cond/uncond sequence 4224 + 4128 "
+                  "tokens, width 3840, 30x128 heads, SwiGLU 10240, adaLN + sandwich norm")
+
+
+def build_block(torch, Z, device, seed=99):
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    bf = lambda *s: (torch.randn(*s, generator=g, device=device) * 0.02).to(torch.bfloat16)
+    nrm = lambda n: 1.0 + 0.1 * torch.randn(n, generator=g, device=device)
+    t = {"w_qkv": bf(3 * D, D), "w_out": bf(D, D), "w_gate_up": bf(2 * F, D), "w_down": bf(D, F),
+         "n_attn": nrm(D), "n_attn_post": nrm(D), "n_ffn": nrm(D), "n_ffn_post": nrm(D),
+         "w_ada": bf(4 * D, E), "b_ada": torch.randn(4 * D, generator=g, device=device) * 0.02}
+    return Z.DeviceBlock.from_tensors(t)
+
+
+def build_model(torch, Z, device, seed=1234):
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    bf = lambda *s: (torch.randn(*s, generator=g, device=device) * 0.02).to(torch.bfloat16)
+    f32 = lambda *s: torch.randn(*s, generator=g, device=device) * 0.02
+    nrm = lambda n: 1.0 + 0.1 * torch.randn(n, generator=g, device=device)
+    blocks = []
+    for kind in KINDS:
+        t = {"w_qkv": bf(3 * D, D), "w_out": bf(D, D), "w_gate_up": bf(2 * F, D), "w_down": bf(D, F),
+             "n_attn": nrm(D), "n_attn_post": nrm(D), "n_ffn": nrm(D), "n_ffn_post": nrm(D)}
+        if kind != "context":
+            t["w_ada"] = bf(4 * D, E)
+            t["b_ada"] = f32(4 * D)
+        blocks.append(Z.DeviceBlock.from_tensors(t))
+    W = {"w_x": bf(D, PATCH), "b_x": f32(D), "w_capnorm": nrm(CAP), "w_cap": bf(D, CAP), "b_cap": f32(D),
+         "pad_vec": torch.randn(D, generator=g, device=device), "w_t1": bf(E, E), "b_t1": f32(E),
+         "w_t2": bf(E, E), "b_t2": f32(E), "w_fada": bf(D, E), "b_fada": f32(D), "w_final": bf(PATCH, D),
+         "b_final": f32(PATCH)}
+    dims = Z.Dims()
+    return Z.DeviceStack(W, dims, 2, 2, 30, patch_dim=PATCH, cap_dim=CAP, blocks=blocks)
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import stream_diffusion_transformer_s3_b200 as Z
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+
+    n_img = GRID[0] * GRID[1]
+    g = torch.Generator(device="cpu")
+    g.manual_seed(42)
+    if args.workload == "stack":
+        stack = build_model(torch, Z, device)
+        # latent noise N(0, 1), 16 x 128 x 128, kept in patch-token layout [4096, 64]
+        latent = torch.randn(16, 128, 128, generator=g).to(device)
+        z = torch.empty(n_img, PATCH, device=device)
+        Z.zdit_patchify(latent, z)
+        caps = torch.randn(sum(N_VALIDS), CAP, generator=g).to(device)
+        call = Z.StackCall(GRID, N_CAPS, N_VALIDS, [0.0, 0.0], z, caps, shared_patches=True)
+        ws = torch.empty(Z.stack_workspace_bytes(stack, call), dtype=torch.uint8, device=device)
+        out = torch.empty(2, n_img, PATCH, device=device)
+        sig = Z.zdit_sigma_schedule(8)
+        inputs = [z, caps]   # per-step inputs (e2e copies them in) ...
+        result = z           # ... and the per-step result copied out
+        flops = forward_flops()
+
+        def step(i):
+            s0, s1 = sig[i % 8], sig[i % 8 + 1]
+            call.set_t([1.0 - s0, 1.0 - s0])
+            Z.zdit_stack_forward(stack, call, out, ws)
+            Z.zdit_euler_cfg_step(z, out[0], out[1], 1.0, s0, s1)
+    else:
+        # one main block of the workload: the joint cond/uncond sequence (4224 + 4128)
+        from stream_diffusion_transformer_s3_b200 import synth
+        blk = build_block(torch, Z, device)
+        lens = [n_img + c for c in N_CAPS]
+        vl = Z.DeviceVarlen([0, lens[0], lens[0] + lens[1]], device=device)
+        T = vl.total
+        x = torch.randn(T, D, generator=g).to(device)
+        temb = torch.randn(2, E, generator=g).to(device)
+        pos = torch.from_numpy(synth.joint_positions(GRID[0], GRID[1], list(N_CAPS))).to(device)
+        cs = torch.empty(T, HD // 2, device=device)
+        sn = torch.empty_like(cs)
+        dims = Z.Dims()
+        Z.zdit_rope_table(pos, dims.rope_axes, dims.rope_theta, cs, sn)
+        fl = Z.flags_of()
+        ws = torch.empty(Z.block_workspace_bytes(dims, fl, T, 2), dtype=torch.uint8, device=device)
+        inputs, result = [x], x
+        flops = 2.0 * T * D * (3 * D + D + 3 * F) + sum(4.0 * D * L * L for L in lens)
+
+        def step(i):
+            Z.zdit_block_forward(dims, fl, blk, vl, x, temb, cs, sn, ws)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if Z.zdit_device_status() != 0:
+        raise RuntimeError("device error during warm-up")
+
+    uuid = str(torch.cuda.get_device_properties(device).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
+    time.sleep(0.3)
+    stream = torch.cuda.current_stream()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    Z.zdit_profile_begin(65536)
+    launches0 = Z.zdit_launch_count()
+    barrier()
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    launches = Z.zdit_launch_count() - launches0
+    kernels = Z.zdit_profile_end()
+    clocks = sampler.stop()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    if Z.zdit_device_status() != 0:
+        raise RuntimeError("device error during the timed region")
+
+    # end to end: pinned host inputs in, result out, every step
+    h_in = [t.cpu().pin_memory() for t in inputs]
+    h_out = torch.empty(result.shape, pin_memory=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        for dst, src in zip(inputs, h_in):
+            dst.copy_(src, non_blocking=True)
+        step(i)
+        h_out.copy_(result, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_e2e = e0.elapsed_time(e1) / args.steps
+
+    if world > 1:
+        t = torch.tensor([ms, ms_e2e], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, ms_e2e = float(t[0]), float(t[1])
+    value = world * flops / (ms * 1e-3) / 1e12
+    value_e2e = world * flops / (ms_e2e * 1e-3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    # a timed region of a few seconds or more runs under the power cap: compare with
+    # the sustained GEMM peak; a short region with the burst peak
+    long_region = ms * args.steps > 3000.0
+    peak_kind = "sustained" if long_region else "burst"
+    peak = peaks["bf16_tflops_sustained"] if long_region else peaks["bf16_tflops"]
+    dom = max(kernels.items(), key=lambda kv: kv[1]["total_ms"]) if kernels else None
+    roofline = None
+    if dom is not None:
+        name, k = dom
+        if k["flops"] > 0:
+            achieved = k["flops"] / (k["total_ms"] * 1e-3) / 1e12
+            roofline = {"kernel": name, "bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+                        "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                        "peak_source": f"{peak_src} bf16 {peak_kind}", "traffic": args.traffic,
+                        "launches_per_step": k["launches"] / args.steps,
+                        "ms_per_launch": k["total_ms"] / k["launches"]}
+    kern_summary = {}
+    total_k = sum(v["total_ms"] for v in kernels.values()) or 1.0
+    for n, k in sorted(kernels.items(), key=lambda kv: -kv[1]["total_ms"]):
+        row = {"launches": k["launches"], "ms_per_step": round(k["total_ms"] / args.steps, 3),
+               "share": round(k["total_ms"] / total_k, 4)}
+        if k["flops"] > 0:
+            row["tflops"] = round(k["flops"] / (k["total_ms"] * 1e-3) / 1e12, 1)
+        if k["bytes"] > 0:
+            row["gbs"] = round(k["bytes"] / (k["total_ms"] * 1e-3) / 1e9, 1)
+        kern_summary[n] = row
+
+    if rank == 0:
+        res = {
+            "metric": "DiT forward TFLOP/s (1024^2, 34-block step, bf16, 1 B200)",
+            "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD if args.workload == "stack" else BLOCK_WORKLOAD,
+                       "global_batch": 2 * world, "seq_len": [n_img + c for c in N_CAPS],
+                       "flops_per_forward": flops, "parallelism": f"replicas x{world}",
+                       "l2": "working set larger than L2 (12.3 GB of bf16 weights streamed per step)",
+                       "frac_of_peak": round(value / world / peak, 4), "peak_kind": peak_kind},
+            "roofline": roofline,
+            "kernels": kern_summary,
+            "gpu_launches": launches,
+            "clocks": clocks,
+            "e2e": {"value": round(value_e2e, 2), "unit": "TFLOP/s", "ms_per_step": round(ms_e2e, 3),
+                    "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in h_in),
+                    "d2h_bytes_per_step": h_out.numel() * h_out.element_size()},
+        }
+        if args.workload == "block":
+            res["metric"] = "DiT main-block forward TFLOP/s (1024^2 cond/uncond sequence, bf16, 1 B200)"
+        if world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline_block(seconds=None)
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ CPU oracle leg
+def _oracle_sample():
+    """One full-width main block of the workload on its uncond branch (L = 4128)."""
+    import numpy as np
+    from stream_diffusion_transformer_s3_b200 import synth
+    case = synth.block_case(11, synth.FULL, GRID[0], GRID[1], [N_CAPS[1]], [N_VALIDS[1]])
+    L = GRID[0] * GRID[1] + N_CAPS[1]
+    flops = 2.0 * L * D * (3 * D + D + 3 * F) + 4.0 * D * L * L
+    return case, flops
+
+
+def _cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"), default=0)
+        if n:
+            return int(n)
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def cpu_baseline_block(seconds=None):
+    import oracle as O
+    case, flops = _oracle_sample()
+    t0 = time.perf_counter()
+    O.block_forward(case["x"], case["cu_seqlens"], case["pos"], case["temb"], case["weights"],
+                    __import__("stream_diffusion_transformer_s3_b200.synth", fromlist=["FULL"]).FULL)
+    dt = time.perf_counter() - t0
+    return {"value": round(flops / dt / 1e12, 5), "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
+            "sample": f"one full-width main block of the workload on its uncond branch (L=4128 tokens), "
+                      f"NumPy float64 oracle, {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle as O
+    from stream_diffusion_transformer_s3_b200 import synth
+    case, flops = _oracle_sample()
+    times = []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        O.block_forward(case["x"], case["cu_seqlens"], case["pos"], case["temb"], case["weights"], synth.FULL)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    sec = sum(times) / len(times)
+    value = flops / sec / 1e12
+    sample = ("each step: one full-width main block of the workload on its uncond branch (L=4128 tokens), "
+              "NumPy float64 oracle on the host cores")
+    res = {"metric": "DiT forward TFLOP/s (1024^2, 34-block step, bf16, 1 B200)", "impl": "reference",
+           "value": round(value, 5), "unit": "TFLOP/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sec * 1e3, 1),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic", "config": {"workload": WORKLOAD, "sample": sample},
+           "cpu_baseline": {"value": round(value, 5), "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": round(value, 5), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=["stack", "block"], default="stack",
+                    help="stack: the full DiT step (default); block: one main block (for kernel captures)")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="dram bytes per launch of the dominant kernel from an ncu capture")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -214,6 +214,9 @@ typedef struct {
   const float* patches;     /* device fp32 [B, n_img, patch_dim] patch tokens  */
   const float* cap_feats;   /* device fp32 [sum n_valid, cap_dim], branches concatenated */
   const float* t;           /* host [B] timestep fed to the DiT (t = 1 - sigma) */
+  int32_t shared_patches;   /* 1: every branch reads the same [n_img, patch_dim]
+                               tokens at `patches` (cond and uncond of one latent);
+                               0: patches holds [B, n_img, patch_dim]           */
 } zdit_stack_inputs;
 
 ZDIT_API size_t zdit_stack_workspace_bytes(const zdit_stack_cfg* cfg, const zdit_stack_inputs* in);
@@ -275,6 +278,30 @@ ZDIT_API zdit_status zdit_patchify(const float* latent, float* tokens, int32_t c
                                    int32_t width, void* stream);
 ZDIT_API zdit_status zdit_unpatchify(const float* tokens, float* latent, int32_t channels, int32_t height,
                                      int32_t width, void* stream);
+
+/* Per-kernel timing of the library's own launches.
+ * zdit_profile_begin(max_records) turns recording on: every kernel launch of the
+ * library is bracketed by two CUDA events on the stream it is launched on (at most
+ * max_records launches are recorded; later ones are counted but not timed).
+ * zdit_profile_end waits for the recorded events, turns recording off and writes
+ * one entry per kernel kind that ran (at most max_entries, which must be >= 16):
+ * its name, launch count, summed event time in ms, summed algorithmic FLOPs
+ * (2 M N K for a GEMM, 4 * 128 * H * sum L^2 for attention) and summed algorithmic
+ * DRAM bytes (each input read once, each output written once).  Host-only
+ * bookkeeping plus cudaEventRecord; intended for benchmarks, not for CUDA-graph
+ * capture.  Errors: ZDIT_ERR_INVALID_ARG, ZDIT_ERR_CUDA. */
+typedef struct {
+  char name[40];
+  int32_t launches;
+  double total_ms;
+  double flops;
+  double bytes;
+} zdit_profile_entry;
+ZDIT_API zdit_status zdit_profile_begin(int32_t max_records);
+ZDIT_API zdit_status zdit_profile_end(zdit_profile_entry* entries, int32_t max_entries, int32_t* n_entries);
+
+/* Number of kernel launches issued by the library since it was loaded. */
+ZDIT_API int64_t zdit_launch_count(void);
 
 /* Synchronizes `stream`, then returns (and clears) the first device-side error
  * latched by any kernel of this library (ZDIT_ERR_DEVICE_TIMEOUT), or

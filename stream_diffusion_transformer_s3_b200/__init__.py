@@ -62,10 +62,19 @@ class StackWeights(C.Structure):
 class StackInputs(C.Structure):
     _fields_ = [("batch", C.c_int32), ("grid_h", C.c_int32), ("grid_w", C.c_int32),
                 ("n_cap", C.POINTER(C.c_int32)), ("n_valid", C.POINTER(C.c_int32)),
-                ("patches", C.c_void_p), ("cap_feats", C.c_void_p), ("t", C.POINTER(C.c_float))]
+                ("patches", C.c_void_p), ("cap_feats", C.c_void_p), ("t", C.POINTER(C.c_float)),
+                ("shared_patches", C.c_int32)]
+
+
+class ProfileEntry(C.Structure):
+    _fields_ = [("name", C.c_char * 40), ("launches", C.c_int32), ("total_ms", C.c_double),
+                ("flops", C.c_double), ("bytes", C.c_double)]
 
 
 _SIGS = {
+    "zdit_profile_begin": (C.c_int, [C.c_int32]),
+    "zdit_profile_end": (C.c_int, [C.POINTER(ProfileEntry), C.c_int32, C.POINTER(C.c_int32)]),
+    "zdit_launch_count": (C.c_int64, []),
     "zdit_version": (C.c_int32, []),
     "zdit_status_string": (C.c_char_p, [C.c_int]),
     "zdit_block_workspace_bytes": (C.c_size_t, [C.POINTER(BlockCfg), C.c_int64, C.c_int32]),
@@ -285,7 +294,7 @@ class DeviceStack:
 class StackCall:
     """Inputs of one zdit_stack_forward call (host arrays kept alive)."""
 
-    def __init__(self, grid, n_caps, n_valids, t, patches, cap_feats):
+    def __init__(self, grid, n_caps, n_valids, t, patches, cap_feats, shared_patches=False):
         B = len(n_caps)
         self.n_cap = (C.c_int32 * B)(*[int(v) for v in n_caps])
         self.n_valid = (C.c_int32 * B)(*[int(v) for v in n_valids])
@@ -294,7 +303,7 @@ class StackCall:
         self.struct = StackInputs(B, int(grid[0]), int(grid[1]), self.n_cap, self.n_valid,
                                   C.c_void_p(patches.data_ptr()),
                                   C.c_void_p(cap_feats.data_ptr()) if cap_feats is not None else None,
-                                  self.t)
+                                  self.t, 1 if shared_patches else 0)
 
     def set_t(self, t):
         for i, v in enumerate(t):
@@ -309,3 +318,21 @@ def zdit_stack_forward(stack: DeviceStack, call: StackCall, out, workspace, stre
     _check(lib().zdit_stack_forward(C.byref(stack.cfg), C.byref(stack.wstruct), C.byref(call.struct),
                                     _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
                                     _stream(stream)), "zdit_stack_forward")
+
+
+def zdit_profile_begin(max_records: int = 65536):
+    _check(lib().zdit_profile_begin(max_records), "zdit_profile_begin")
+
+
+def zdit_profile_end() -> dict:
+    """{kernel kind: {launches, total_ms, flops, bytes}} of the launches recorded
+    since zdit_profile_begin."""
+    buf = (ProfileEntry * 32)()
+    n = C.c_int32(0)
+    _check(lib().zdit_profile_end(buf, 32, C.byref(n)), "zdit_profile_end")
+    return {buf[i].name.decode(): {"launches": buf[i].launches, "total_ms": buf[i].total_ms,
+                                   "flops": buf[i].flops, "bytes": buf[i].bytes} for i in range(n.value)}
+
+
+def zdit_launch_count() -> int:
+    return int(lib().zdit_launch_count())

@@ -141,7 +141,7 @@ zdit_status run_block(const zdit_block_cfg& cfg, const zdit_block_weights& w, co
   GemmArgs g{};
   g.A = ws.a; g.lda = D; g.B = w.w_qkv; g.ldb = D; g.M = T; g.N = 3 * D; g.K = D;
   g.epi = EPI_QKV; g.out = ws.qkvh; g.ldo = 3 * D; g.rope_cos = rcos; g.rope_sin = rsin; g.dim = D;
-  g.qn = qkn ? w.n_q : nullptr; g.kn = qkn ? w.n_k : nullptr; g.eps = cfg.norm_eps;
+  g.prof_kind = PROF_GEMM_QKV; g.qn = qkn ? w.n_q : nullptr; g.kn = qkn ? w.n_k : nullptr; g.eps = cfg.norm_eps;
   zdit_status st = launch_gemm(g, s);
   if (st != ZDIT_OK) return st;
 
@@ -157,7 +157,7 @@ zdit_status run_block(const zdit_block_cfg& cfg, const zdit_block_weights& w, co
   // output projection -> y fp32
   GemmArgs go{};
   go.A = ws.o; go.lda = D; go.B = w.w_out; go.ldb = D; go.M = T; go.N = D; go.K = D;
-  go.epi = EPI_F32; go.out = ws.y; go.ldo = D;
+  go.epi = EPI_F32; go.out = ws.y; go.ldo = D; go.prof_kind = PROF_GEMM_OUT;
   st = launch_gemm(go, s);
   if (st != ZDIT_OK) return st;
 
@@ -172,14 +172,14 @@ zdit_status run_block(const zdit_block_cfg& cfg, const zdit_block_weights& w, co
   // gate/up projection with SwiGLU epilogue -> h bf16 [T, F]
   GemmArgs gu{};
   gu.A = ws.a; gu.lda = D; gu.B = w.w_gate_up; gu.ldb = D; gu.M = T; gu.N = 2 * F; gu.K = D;
-  gu.epi = EPI_SWIGLU; gu.out = ws.qkvh; gu.ldo = F;
+  gu.epi = EPI_SWIGLU; gu.out = ws.qkvh; gu.ldo = F; gu.prof_kind = PROF_GEMM_GATE_UP;
   st = launch_gemm(gu, s);
   if (st != ZDIT_OK) return st;
 
   // down projection -> y fp32
   GemmArgs gd{};
   gd.A = ws.qkvh; gd.lda = F; gd.B = w.w_down; gd.ldb = F; gd.M = T; gd.N = D; gd.K = F;
-  gd.epi = EPI_F32; gd.out = ws.y; gd.ldo = D;
+  gd.epi = EPI_F32; gd.out = ws.y; gd.ldo = D; gd.prof_kind = PROF_GEMM_DOWN;
   st = launch_gemm(gd, s);
   if (st != ZDIT_OK) return st;
 
@@ -401,7 +401,9 @@ ZDIT_API zdit_status zdit_stack_forward(const zdit_stack_cfg* cfg, const zdit_st
   launch_gemv(static_cast<const __nv_bfloat16*>(w->w_fada), w->b_fada, ws.temb, B, E, D, ws.fmod, s);
 
   // image embedder: patches -> bf16 -> Linear(patch_dim, D) + bias
-  launch_cast_bf16(in->patches, ws.patches16, (int64_t)d.T_img * d.patch_dim, s);
+  for (int b = 0; b < B; ++b)
+    launch_cast_bf16(in->patches + (in->shared_patches ? 0 : (size_t)b * d.n_img * d.patch_dim),
+                     ws.patches16 + (size_t)b * d.n_img * d.patch_dim, (int64_t)d.n_img * d.patch_dim, s);
   GemmArgs gx{};
   gx.A = ws.patches16; gx.lda = d.patch_dim; gx.B = w->w_x; gx.ldb = d.patch_dim; gx.M = d.T_img; gx.N = D;
   gx.K = d.patch_dim; gx.epi = EPI_F32; gx.out = ws.x_img; gx.ldo = D; gx.bias = w->b_x;

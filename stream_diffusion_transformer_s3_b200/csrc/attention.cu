@@ -344,6 +344,12 @@ zdit_status launch_attention(const AttnArgs& a, cudaStream_t s) {
   p.cu = a.cu_seqlens_dev;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.err = device_error_ptr();
+  double l2 = 0.0;
+  for (int b = 0; b < a.batch; ++b) {
+    const double L = a.cu_seqlens_host[b + 1] - a.cu_seqlens_host[b];
+    l2 += L * L;
+  }
+  ProfScope ps(PROF_ATTENTION, 4.0 * HD * a.n_heads * l2, 4.0 * 2.0 * a.T * (double)cols, s);
   dim3 grid(total_qt, a.n_heads);
   attn_tc_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? ZDIT_OK : ZDIT_ERR_CUDA;

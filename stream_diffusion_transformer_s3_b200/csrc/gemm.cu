@@ -376,6 +376,10 @@ zdit_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
   kp.group_m = 16;
   kp.err = device_error_ptr();
   const int tiles = kp.num_m * kp.num_n;
+  const double out_elt = (a.epi == EPI_F32) ? 4.0 : 2.0;
+  const double out_cols = (a.epi == EPI_SWIGLU) ? a.N / 2.0 : (double)a.N;
+  ProfScope ps(a.prof_kind, 2.0 * a.M * a.N * (double)a.K,
+               2.0 * ((double)a.M * a.K + (double)a.N * a.K) + out_elt * a.M * out_cols, s);
   const int grid = tiles < num_sms() ? tiles : num_sms();
   switch (a.epi) {
     case EPI_F32: return launch_epi<EPI_F32>(ta, tb, kp, grid, s);

@@ -9,6 +9,30 @@
 
 namespace zdit {
 
+// ---------------------------------------------------------------- launch accounting
+enum ProfKind : int {
+  PROF_GEMM_QKV = 0, PROF_GEMM_OUT, PROF_GEMM_GATE_UP, PROF_GEMM_DOWN, PROF_GEMM_OTHER,
+  PROF_ATTENTION, PROF_NORM_MOD, PROF_RESIDUAL, PROF_GEMV, PROF_EULER, PROF_ROPE, PROF_MISC,
+  PROF_NUM_KINDS
+};
+
+// Counts one kernel launch; when profiling is on, brackets it with CUDA events on
+// stream `s` (construct just before the launch, destroy just after).
+class ProfScope {
+ public:
+  ProfScope(int kind, double flops, double bytes, cudaStream_t s);
+  ~ProfScope();
+  ProfScope(const ProfScope&) = delete;
+  ProfScope& operator=(const ProfScope&) = delete;
+
+ private:
+  int kind_;
+  double flops_, bytes_;
+  cudaStream_t s_;
+  cudaEvent_t a_ = nullptr, b_ = nullptr;
+  bool active_ = false;
+};
+
 // ---------------------------------------------------------------- GEMM (tcgen05)
 // C[M, N] = A[M, K] . B[N, K]^T with bf16 A, B (both K-major, row-major in memory)
 // and an fp32 accumulator in TMEM, followed by one of the fused epilogues.
@@ -33,6 +57,7 @@ struct GemmArgs {
   const float* qn;        // [128] per-head RMSNorm weights (EPI_QKV, optional)
   const float* kn;
   float eps;
+  int prof_kind = PROF_GEMM_OTHER;
 };
 
 zdit_status launch_gemm(const GemmArgs& a, cudaStream_t s);

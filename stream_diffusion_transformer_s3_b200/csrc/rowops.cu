@@ -411,6 +411,7 @@ __global__ void stack_layout_kernel(LayoutParams lp, int* __restrict__ pos_img, 
 
 void launch_stack_layout(const int* n_cap, int B, int grid_h, int grid_w, int* pos_img, int* pos_cap, int* pos_joint,
                          int* cu_img, int* cu_cap, int* cu_joint, cudaStream_t s) {
+  ProfScope ps(PROF_MISC, 0.0, 0.0, s);
   LayoutParams lp;
   lp.B = B; lp.grid_h = grid_h; lp.grid_w = grid_w;
   int64_t T = 0;
@@ -425,6 +426,7 @@ void launch_stack_layout(const int* n_cap, int B, int grid_h, int grid_w, int* p
 void launch_norm_modulate_ex(const float* x, int T, int D, const float* w, const float* mod, int mod_stride,
                              const int* cu, int batch, int fixed_branch, int layer_norm, float eps,
                              __nv_bfloat16* out, cudaStream_t s) {
+  ProfScope ps(PROF_NORM_MOD, 0.0, (double)T * D * (4.0 + 2.0), s);
   NormModParams p{x, D, w, mod, mod_stride, cu, batch, fixed_branch, layer_norm, eps, out};
   const int v = (D + RT * 4 - 1) / (RT * 4);
   if (T <= 0) return;
@@ -443,6 +445,7 @@ void launch_norm_modulate(const RowModArgs& a, cudaStream_t s) {
 }
 
 void launch_residual(const ResidArgs& a, cudaStream_t s) {
+  ProfScope ps(PROF_RESIDUAL, 0.0, (double)a.T * a.D * (12.0 + (a.next_out ? 2.0 : 0.0)), s);
   ResidParams p{a.x,       a.y,    a.D,          a.post_w,  a.gate,       a.gate_stride, a.tanh_gate,
                 a.cu_seqlens, a.batch, a.eps,    a.next_w,  a.next_scale, a.next_scale_stride, a.next_out};
   const int v = (a.D + RT * 4 - 1) / (RT * 4);
@@ -459,10 +462,12 @@ void launch_residual(const ResidArgs& a, cudaStream_t s) {
 
 void launch_gemv(const __nv_bfloat16* W, const float* bias, const float* temb, int B, int E, int rows, float* out,
                  cudaStream_t s) {
+  ProfScope ps(PROF_GEMV, 2.0 * rows * (double)E * B, 2.0 * rows * (double)E + 4.0 * rows * (B + 1.0), s);
   adaln_gemv_kernel<<<(rows + 7) / 8, 256, (size_t)B * E * sizeof(float), s>>>(W, bias, temb, B, E, rows, out);
 }
 
 void launch_euler_cfg(float* x, const float* vp, const float* vn, int64_t n, float g, float dsig, cudaStream_t s) {
+  ProfScope ps(PROF_EULER, 0.0, 4.0 * (double)n * (vn != nullptr ? 4.0 : 3.0), s);
   int blocks = (int)((n / 4 + 255) / 256);
   if (blocks < 1) blocks = 1;
   if (blocks > 4 * num_sms()) blocks = 4 * num_sms();
@@ -471,6 +476,7 @@ void launch_euler_cfg(float* x, const float* vp, const float* vn, int64_t n, flo
 
 void launch_rope_table(const int* pos, int64_t T, int head_dim, const int* axes, float theta, float* cs, float* sn,
                        cudaStream_t s) {
+  ProfScope ps(PROF_ROPE, 0.0, 8.0 * (double)T * (head_dim / 2) + 12.0 * T, s);
   const int64_t n = T * (head_dim / 2);
   if (n <= 0) return;
   rope_table_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(pos, T, head_dim / 2, axes[0], axes[1], axes[2],
@@ -479,23 +485,27 @@ void launch_rope_table(const int* pos, int64_t T, int head_dim, const int* axes,
 
 void launch_timestep_embed(const float* t_host, int B, int E, float t_scale, const __nv_bfloat16* w1,
                            const float* b1, const __nv_bfloat16* w2, const float* b2, float* temb, cudaStream_t s) {
+  ProfScope ps(PROF_MISC, 0.0, 0.0, s);
   TembParams tp;
   for (int i = 0; i < 8; ++i) tp.t[i] = i < B ? t_host[i] : 0.f;
   timestep_embed_kernel<<<B, 256, 2 * E * sizeof(float), s>>>(tp, E, t_scale, w1, b1, w2, b2, temb);
 }
 
 void launch_patchify(const float* src, float* dst, int C, int h, int w, int dir, cudaStream_t s) {
+  ProfScope ps(PROF_MISC, 0.0, 8.0 * (double)h * w * 4 * C, s);
   const int64_t total = (int64_t)h * w * 4 * C;
   if (total <= 0) return;
   patchify_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(src, dst, C, h, w, dir);
 }
 
 void launch_cast_bf16(const float* src, __nv_bfloat16* dst, int64_t n, cudaStream_t s) {
+  ProfScope ps(PROF_MISC, 0.0, 6.0 * (double)n, s);
   if (n <= 0) return;
   cast_bf16_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(src, dst, n);
 }
 
 void launch_fill_rows(float* x, int D, int nrows, const float* vec, cudaStream_t s) {
+  ProfScope ps(PROF_MISC, 0.0, 4.0 * (double)nrows * D, s);
   const int64_t n = (int64_t)nrows * D;
   if (n <= 0) return;
   fill_rows_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(x, D, nrows, vec);
