@@ -295,7 +295,7 @@ def run_ours(args):
             "config": {"workload": WORKLOAD if args.workload == "stack" else BLOCK_WORKLOAD,
                        "global_batch": 2 * world, "seq_len": [n_img + c for c in N_CAPS],
                        "flops_per_forward": flops, "parallelism": f"replicas x{world}",
-                       "l2": "working set larger than L2 (12.3 GB of bf16 weights streamed per step)",
+                       "l2": ("working set larger than L2 (12.3 GB of bf16 weights streamed per step)" if args.workload == "stack" else "working set larger than L2 (354 MB weights + 128 MB residual + 448 MB activations per block)"),
                        "frac_of_peak": round(value / world / peak, 4), "peak_kind": peak_kind},
             "roofline": roofline,
             "kernels": kern_summary,
