@@ -160,6 +160,31 @@ ZDIT_API zdit_status zdit_block_forward(const zdit_block_cfg* cfg, const zdit_bl
                                         const float* rope_cos, const float* rope_sin, void* workspace,
                                         size_t workspace_bytes, void* stream);
 
+/* zdit_block_forward without a caller workspace, for callers that cannot allocate
+ * device memory: a plugin running inside a host framework that has already reserved
+ * (nearly) all of the GPU for its own pool, so cudaMalloc would fail, or a
+ * latency-critical loop that must not pay cudaMalloc's device-wide synchronization.
+ * The pages describe no such entry point; it has no counterpart there.
+ *   Same arguments and result as zdit_block_forward, minus the workspace.  The
+ *   workspace is a 40 MiB device array owned by the library (held on every GPU that
+ *   loads the library until the process exits); calls needing more than 40 MiB of
+ *   workspace (zdit_block_workspace_bytes) return ZDIT_ERR_WORKSPACE and launch
+ *   nothing.  At full width (D 3840, F 10240, two branches) that admits up to 777 tokens,
+ *   e.g. the 256px cond/uncond pair (608 tokens).
+ *   The call allocates nothing (no cudaMalloc, cudaFree or allocating library call).
+ *   The first call on a device looks up the array's device address (once per
+ *   device, with that device current); make that first call before any stream
+ *   capture.
+ *   All calls share the one array and it keeps the previous call's contents (the
+ *   block writes every workspace byte it reads, so nothing needs clearing): calls
+ *   whose execution overlaps on the GPU (different streams, or host threads) race
+ *   on it and must be serialized by the caller.
+ * Errors: as zdit_block_forward, plus ZDIT_ERR_WORKSPACE (too many tokens) and
+ * ZDIT_ERR_CUDA (address lookup failed). */
+ZDIT_API zdit_status zdit_block_forward_static(const zdit_block_cfg* cfg, const zdit_block_weights* w,
+                                               const zdit_varlen* varlen, float* x, const float* temb,
+                                               const float* rope_cos, const float* rope_sin, void* stream);
+
 /* Whole DiT. */
 typedef struct {
   zdit_block_cfg block;      /* shared by all blocks; ADALN is dropped for the

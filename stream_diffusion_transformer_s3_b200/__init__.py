@@ -81,6 +81,8 @@ _SIGS = {
     "zdit_block_forward": (C.c_int, [C.POINTER(BlockCfg), C.POINTER(BlockWeights), C.POINTER(Varlen),
                                      C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
                                      C.c_size_t, C.c_void_p]),
+    "zdit_block_forward_static": (C.c_int, [C.POINTER(BlockCfg), C.POINTER(BlockWeights), C.POINTER(Varlen),
+                                            C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
     "zdit_stack_workspace_bytes": (C.c_size_t, [C.POINTER(StackCfg), C.POINTER(StackInputs)]),
     "zdit_stack_forward": (C.c_int, [C.POINTER(StackCfg), C.POINTER(StackWeights), C.POINTER(StackInputs),
                                      C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]),
@@ -221,6 +223,16 @@ def zdit_block_forward(dims: Dims, flags: int, weights: DeviceBlock, varlen: Dev
                                     _ptr(temb), _ptr(rope_cos), _ptr(rope_sin), _ptr(workspace),
                                     workspace.numel() * workspace.element_size(), _stream(stream))
     _check(code, "zdit_block_forward")
+
+
+def zdit_block_forward_static(dims: Dims, flags: int, weights: DeviceBlock, varlen: DeviceVarlen, x, temb,
+                              rope_cos, rope_sin, stream=None):
+    """zdit_block_forward with the library's static 40 MiB scratch as workspace: for
+    callers that cannot allocate device memory.  Calls must not overlap on the GPU."""
+    c = dims.cfg(flags)
+    code = lib().zdit_block_forward_static(C.byref(c), C.byref(weights.struct), C.byref(varlen.struct), _ptr(x),
+                                           _ptr(temb), _ptr(rope_cos), _ptr(rope_sin), _stream(stream))
+    _check(code, "zdit_block_forward_static")
 
 
 def zdit_rope_table(pos, rope_axes, theta, cos_out, sin_out, head_dim=128, stream=None):

@@ -1,0 +1,66 @@
+"""zdit_block_forward_static: the block forward for callers that cannot allocate
+device memory (a plugin whose host framework has reserved the GPU's memory for its
+own pool, or a loop that must not pay cudaMalloc's device-wide synchronization).
+
+Checks, through the C ABI on the GPU, that two calls in a row (sharing the library's
+static scratch) give the same block output as zdit_block_forward with a caller
+workspace, within the block-parity tolerance, and that a call too large for the
+40 MiB scratch is refused before any launch.  This file is collected last."""
+import ctypes as C
+
+import numpy as np
+import pytest
+import torch
+
+import stream_diffusion_transformer_s3_b200 as Z
+from stream_diffusion_transformer_s3_b200 import synth
+from _gpu import dev, dims_of, errors, host, require_gpu, rope_tables
+
+pytestmark = pytest.mark.gpu
+TOL = 2e-2
+
+
+@pytest.fixture(autouse=True)
+def _gpu():
+    require_gpu()
+
+
+def test_static_scratch_block_matches_workspace_block_twice():
+    case = synth.config2(0)  # full width, cond/uncond 320 + 288 tokens (31.3 MiB of scratch)
+    d = synth.FULL
+    dims = dims_of(d)
+    fl = Z.flags_of()
+    w = Z.DeviceBlock(case["weights"])
+    vl = Z.DeviceVarlen(case["cu_seqlens"])
+    temb = dev(case["temb"])
+    cs, sn = rope_tables(case["pos"], dims)
+
+    x_ref = dev(case["x"])
+    ws = torch.empty(Z.block_workspace_bytes(dims, fl, vl.total, 2), dtype=torch.uint8, device="cuda")
+    Z.zdit_block_forward(dims, fl, w, vl, x_ref, temb, cs, sn, ws)
+    assert Z.zdit_device_status() == 0
+    ref = host(x_ref)
+    upd_ref = ref - case["x"]
+
+    for _ in range(2):  # the second call finds the first call's data in the scratch
+        x = dev(case["x"])
+        Z.zdit_block_forward_static(dims, fl, w, vl, x, temb, cs, sn)
+        assert Z.zdit_device_status() == 0
+        got = host(x)
+        e_out = errors(got, ref)
+        e_upd = errors(got - case["x"], upd_ref)
+        assert e_out["rel_l2"] <= TOL, e_out
+        assert e_upd["rel_l2"] <= TOL, e_upd
+
+
+def test_static_scratch_refuses_oversized_call():
+    dims = Z.Dims()
+    fl = Z.flags_of()
+    T = 2048  # needs ~105 MiB of workspace at full width
+    assert Z.block_workspace_bytes(dims, fl, T, 2) > (40 << 20)
+    vl = Z.DeviceVarlen([0, 1024, T])
+    cfg = dims.cfg(fl)
+    wts = Z.BlockWeights(**{f: C.c_void_p(1 << 20) for f, _ in Z.BlockWeights._fields_})
+    code = Z.lib().zdit_block_forward_static(C.byref(cfg), C.byref(wts), C.byref(vl.struct), C.c_void_p(1 << 20),
+                                             C.c_void_p(1 << 20), C.c_void_p(1 << 20), C.c_void_p(1 << 20), None)
+    assert code == -4  # ZDIT_ERR_WORKSPACE, nothing launched
