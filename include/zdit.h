@@ -64,12 +64,12 @@ typedef enum {
 /* Block feature flags. */
 enum {
   ZDIT_F_ADALN = 1,         /* adaLN modulation from the timestep embedding; when
-                               clear the block uses scale 0 and gate 1 (context
-                               refiner, [CoreAI] DiT row "no adaLN")            */
+                               clear the block uses scale 0 and gate 1 (the
+                               context refiner has none, [CoreAI] DiT row)      */
   ZDIT_F_SANDWICH_NORM = 2, /* RMSNorm(y) * w_post of each projection output before
-                               its gated add (reading of [Jobs] "... retain FP32
-                               range before normalization" and of the 3.1e5 output
-                               vs 6.7e3 residual ranges in [CoreAI])            */
+                               its gated add (reading of [Jobs]: projection outputs
+                               stay in FP32 range until normalized; and of the
+                               3.1e5 output vs 6.7e3 residual ranges in [CoreAI]) */
   ZDIT_F_QK_NORM = 4,       /* per-head RMSNorm of q and k before RoPE (option) */
   ZDIT_F_TANH_GATE = 8      /* gate = tanh(adaLN gate chunk) (option)           */
 };

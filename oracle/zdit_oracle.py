@@ -143,7 +143,7 @@ def branch_of_token(cu_seqlens):
 def adaln_vectors(temb, w, dim: int, flags: Flags):
     """(scale_attn, gate_attn, scale_ffn, gate_ffn), each [B, D] (R1).
 
-    Without adaLN (context refiner, [CoreAI] DiT row "2 context-refiner (no adaLN)"):
+    Without adaLN (the context refiner has none, [CoreAI] DiT row):
     scale = 0 and gate = 1.
     """
     B = np.asarray(temb).shape[0]
