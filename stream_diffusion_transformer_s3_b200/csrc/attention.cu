@@ -1,17 +1,24 @@
 // Varlen joint attention for sm_100a (head dim 128), flash-style with tcgen05.
 //
-// One CTA computes one (branch, head, 128-row query tile):
+// One CTA computes two 128-row query tiles of one (branch, head):
 //   O = softmax(Q K^T / sqrt(128)) V over all L_b tokens of its branch segment.
 // There is no mask inside a segment: caption pad tokens are ordinary context
 // ("Z-Image-Turbo port", "The three things that each cost a wrong image", item 3),
 // branches never see each other, and only the columns past the segment end of the
 // last key tile are excluded.
 //
-// Warp roles (192 threads):
-//   warp 0 lane 0 : TMA producer (Q once; K and V tiles in separate 2-deep rings)
-//   warp 1 lane 0 : tcgen05.mma issuer (S = Q K^T into TMEM, O += P V from smem P)
-//   warps 2-5     : softmax, one thread per query row (TMEM lane)
-// TMEM columns: S ping-pong at [0,128) and [128,256), O at [256,384).
+// Warp roles (320 threads):
+//   warps 0-3 : softmax of query tile 0, one thread per query row (TMEM lane)
+//   warps 4-7 : softmax of query tile 1
+//   warp 8    : TMA producer (Q0, Q1 once; K and V tiles in separate 2-deep rings)
+//   warp 9    : tcgen05.mma issuer
+// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).  P_t (bf16,
+// two per 32-bit column) is written back over the first 64 columns of S_t and fed
+// to the PV product straight from TMEM, so P never touches shared memory.
+// The tensor core alternates between the two tiles: PV0(j-1), S0(j), PV1(j-1),
+// S1(j), ... so the softmax of one tile overlaps the MMAs of the other.  Because
+// PV_t(j-1) is issued before S_t(j), the commit that signals S_t(j) also proves that
+// PV_t(j-1) is done: the softmax may then overwrite P_t and rescale O_t freely.
 // Online softmax in FP32 with a lazily moved reference max: the running max only
 // moves (and O is rescaled) when a row's max grows by more than 2^8, so the common
 // tile needs no O round trip; P = exp2(s - m_ref) <= 256 stays in bf16 range.
@@ -27,18 +34,17 @@ bool make_tmap_bf16_2d(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t 
 
 namespace {
 
-constexpr int TILE = 128;          // query rows and key rows per tile
-constexpr int HD = 128;            // head dim
+constexpr int TILE = 128;            // query rows and key rows per tile
+constexpr int HD = 128;              // head dim
 constexpr int HALF = TILE * 64 * 2;  // one 64-column swizzled half tile: 16 KB
 constexpr int TILE_BYTES = 2 * HALF;
-constexpr int THREADS = 192;
-constexpr int KV_STAGES = 2;
-// smem: Q | K[2] | V[2] | P, then barriers
+constexpr int THREADS = 320;
+constexpr int WARP_LOAD = 8, WARP_MMA = 9;
+// smem: Q0 | Q1 | K[2] | V[2], then barriers
 constexpr int OFF_Q = 0;
-constexpr int OFF_K = OFF_Q + TILE_BYTES;
-constexpr int OFF_V = OFF_K + KV_STAGES * TILE_BYTES;
-constexpr int OFF_P = OFF_V + KV_STAGES * TILE_BYTES;
-constexpr int OFF_BAR = OFF_P + TILE_BYTES;
+constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
+constexpr int OFF_V = OFF_K + 2 * TILE_BYTES;
+constexpr int OFF_BAR = OFF_V + 2 * TILE_BYTES;
 constexpr int SMEM_BYTES = 1024 + OFF_BAR + 256;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
@@ -63,14 +69,13 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;   // [2]
-  uint64_t* k_empty = bars + 3;  // [2]
-  uint64_t* v_full = bars + 5;   // [2]
-  uint64_t* v_empty = bars + 7;  // [2]
-  uint64_t* s_full = bars + 9;   // [2]
-  uint64_t* s_empty = bars + 11; // [2]
-  uint64_t* p_full = bars + 13;
-  uint64_t* pv_done = bars + 14;
+  uint64_t* k_full = bars + 1;    // [2]
+  uint64_t* k_empty = bars + 3;   // [2]
+  uint64_t* v_full = bars + 5;    // [2]
+  uint64_t* v_empty = bars + 7;   // [2]
+  uint64_t* s_full = bars + 9;    // [2] one per query tile
+  uint64_t* p_full = bars + 11;   // [2]
+  uint64_t* o_full = bars + 13;   // [2]
   uint64_t* mma_done = bars + 15;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -79,19 +84,19 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int lane = threadIdx.x & 31;
   const int head = blockIdx.y;
 
-  // locate (branch, query tile) of this CTA
-  int b = 0, qt = blockIdx.x;
+  // locate (branch, query-tile pair) of this CTA
+  int b = 0, pair = blockIdx.x;
   int seg0 = 0, L = 0;
   for (; b < p.batch; ++b) {
     seg0 = p.cu[b];
     L = p.cu[b + 1] - seg0;
-    const int nq = (L + TILE - 1) / TILE;
-    if (qt < nq) break;
-    qt -= nq;
+    const int np = ((L + TILE - 1) / TILE + 1) / 2;
+    if (pair < np) break;
+    pair -= np;
   }
   if (b >= p.batch) return;  // (grid sized exactly; defensive, uniform per CTA)
   const int n_kv = (L + TILE - 1) / TILE;
-  const int q0 = seg0 + qt * TILE;
+  const int q0 = seg0 + pair * 2 * TILE;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -101,32 +106,33 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 4);
+      mbar_init(&p_full[i], 4);
+      mbar_init(&o_full[i], 1);
     }
-    mbar_init(p_full, 4);
-    mbar_init(pv_done, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 0 && lane == 0) {
+  if (warp == WARP_LOAD && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
   }
-  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  if (warp == WARP_MMA) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int col0 = head * HD;
 
-  if (warp == 0 && lane == 0) {
+  if (warp == WARP_LOAD && lane == 0) {
     // ------------------------------------------------------------ producer
     uint8_t* sQ = smem + OFF_Q;
-    mbar_arrive_expect_tx(q_full, TILE_BYTES);
+    mbar_arrive_expect_tx(q_full, 2 * TILE_BYTES);
     tma_load_2d(sQ, &tmQ, q_full, col0, q0);
     tma_load_2d(sQ + HALF, &tmQ, q_full, col0 + 64, q0);
+    tma_load_2d(sQ + TILE_BYTES, &tmQ, q_full, col0, q0 + TILE);
+    tma_load_2d(sQ + TILE_BYTES + HALF, &tmQ, q_full, col0 + 64, q0 + TILE);
     int nk_issued = 0, nv_issued = 0;
     for (int j = 0; j < n_kv; ++j) {
       const int st = j & 1;
@@ -153,73 +159,81 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int j = (nv_issued > 2 ? nv_issued - 2 : 0); j < nv_issued; ++j)
         mbar_wait(&v_full[j & 1], (j >> 1) & 1, &dummy);
     }
-  } else if (warp == 1 && lane == 0) {
+  } else if (warp == WARP_MMA && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
-    const uint32_t id_s = idesc_bf16_f32(TILE, TILE);                // K-major A and B
-    const uint32_t id_o = idesc_bf16_f32(TILE, HD, false, true);     // B (V) MN-major
+    const uint32_t id_s = idesc_bf16_f32(TILE, TILE);             // Q, K both K-major
+    const uint32_t id_o = idesc_bf16_f32(TILE, HD, false, true);  // P from TMEM, V MN-major
     const uint32_t aQ = smem_u32(smem + OFF_Q);
-    const uint32_t aP = smem_u32(smem + OFF_P);
-    auto issue_pv = [&](int i) -> bool {
-      if (!mbar_wait(p_full, i & 1, abort_flag, p.err)) return false;
-      if (!mbar_wait(&v_full[i & 1], (i >> 1) & 1, abort_flag, p.err)) return false;
+    // O_t += P_t V_i ; P_t read from TMEM columns [t*128, t*128 + 64)
+    auto issue_pv = [&](int t, int i) -> bool {
+      if (!mbar_wait(&p_full[t], i & 1, abort_flag, p.err)) return false;
+      if (t == 0 && !mbar_wait(&v_full[i & 1], (i >> 1) & 1, abort_flag, p.err)) return false;
       tc_fence_after();
       const uint32_t aV = smem_u32(smem + OFF_V + (i & 1) * TILE_BYTES);
 #pragma unroll
-      for (int k = 0; k < TILE / 16; ++k) {
-        const uint64_t ad = sdesc_kmajor_sw128(aP + (k >> 2) * HALF + (k & 3) * 32);
-        const uint64_t bd = sdesc_mnmajor_sw128(aV + k * 16 * 128, HALF, 1024);
-        umma_bf16_ss(tmem + 256, ad, bd, id_o, (i | k) != 0 ? 1u : 0u);
-      }
-      umma_commit(&v_empty[i & 1]);
-      umma_commit(pv_done);
+      for (int k = 0; k < TILE / 16; ++k)
+        umma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + k * 8,
+                     sdesc_mnmajor_sw128(aV + k * 16 * 128, HALF, 1024), id_o, (i | k) != 0 ? 1u : 0u);
       return true;
     };
-    bool ok = mbar_wait(q_full, 0, abort_flag, p.err);
-    for (int j = 0; ok && j < n_kv; ++j) {
-      const int st = j & 1;
-      if (!mbar_wait(&s_empty[st], ((j >> 1) & 1) ^ 1, abort_flag, p.err)) { ok = false; break; }
-      if (!mbar_wait(&k_full[st], (j >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
-      tc_fence_after();
-      const uint32_t aK = smem_u32(smem + OFF_K + st * TILE_BYTES);
+    // S_t = Q_t K_j^T into TMEM columns [t*128, t*128 + 128)
+    auto issue_s = [&](int t, int j) {
+      const uint32_t aK = smem_u32(smem + OFF_K + (j & 1) * TILE_BYTES);
+      const uint32_t aQt = aQ + t * TILE_BYTES;
 #pragma unroll
       for (int k = 0; k < HD / 16; ++k) {
         const uint32_t off = (k >> 2) * HALF + (k & 3) * 32;
-        umma_bf16_ss(tmem + st * TILE, sdesc_kmajor_sw128(aQ + off), sdesc_kmajor_sw128(aK + off), id_s,
+        umma_bf16_ss(tmem + t * 128, sdesc_kmajor_sw128(aQt + off), sdesc_kmajor_sw128(aK + off), id_s,
                      k != 0 ? 1u : 0u);
       }
-      umma_commit(&k_empty[st]);
-      umma_commit(&s_full[st]);
-      if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+      umma_commit(&s_full[t]);
+    };
+    bool ok = mbar_wait(q_full, 0, abort_flag, p.err);
+    for (int j = 0; ok && j < n_kv; ++j) {
+      if (!mbar_wait(&k_full[j & 1], (j >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
+      tc_fence_after();
+      if (j > 0 && !issue_pv(0, j - 1)) { ok = false; break; }
+      issue_s(0, j);
+      if (j > 0) {
+        if (!issue_pv(1, j - 1)) { ok = false; break; }
+        umma_commit(&v_empty[(j - 1) & 1]);
+      }
+      issue_s(1, j);
+      umma_commit(&k_empty[j & 1]);
     }
-    if (ok) issue_pv(n_kv - 1);
+    if (ok && issue_pv(0, n_kv - 1)) {
+      umma_commit(&o_full[0]);
+      if (issue_pv(1, n_kv - 1)) {
+        umma_commit(&o_full[1]);
+        umma_commit(&v_empty[(n_kv - 1) & 1]);
+      }
+    }
     umma_commit(mma_done);
     int dummy = 0;
     mbar_wait(mma_done, 0, &dummy);
-  } else if (warp >= 2) {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ softmax
-    const int lg = warp & 3;
+    const int t = warp >> 2;         // query tile of this warpgroup
+    const int lg = warp & 3;         // TMEM lane group
     const int row = lg * 32 + lane;  // query row inside the tile == TMEM lane
     const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
-    uint8_t* sP = smem + OFF_P;
+    const uint32_t tS = tmem + lane_off + t * 128;
+    const uint32_t tO = tmem + lane_off + 256 + t * 128;
     float m_ref = -INFINITY, l_sum = 0.f;
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
-      const int st = j & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[st], (j >> 1) & 1, abort_flag, p.err));
+      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1, abort_flag, p.err));
       if (!ok) break;
       tc_fence_after();
       float s[TILE];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t r[32];
-        tmem_ld32(tmem + lane_off + st * TILE + c * 32, r);
-        tmem_ld_wait();
+        tmem_ld32(tS + c * 32, r);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(r[e]) * p.scale_log2;
+        for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(r[e]);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_empty[st]);
+      tmem_ld_wait();
       const int valid = L - j * TILE;  // keys past the segment end are excluded
       if (valid < TILE) {
 #pragma unroll
@@ -229,6 +243,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       float mx = -INFINITY;
 #pragma unroll
       for (int e = 0; e < TILE; ++e) mx = fmaxf(mx, s[e]);
+      mx *= p.scale_log2;
       float alpha = 1.f;
       bool move = false;
       if (j == 0) {
@@ -239,57 +254,48 @@ __global__ void __launch_bounds__(THREADS, 1)
         move = true;
       }
       l_sum *= alpha;
-      uint32_t pk[TILE / 2];
-      float part = 0.f;
-#pragma unroll
-      for (int e = 0; e < TILE / 2; ++e) {
-        const float p0 = ex2(s[2 * e] - m_ref);
-        const float p1 = ex2(s[2 * e + 1] - m_ref);
-        part += p0 + p1;
-        pk[e] = pack_bf16x2(p0, p1);
-      }
-      l_sum += part;
-      if (j >= 1) {  // P buffer free and O stable once PV of the previous tile is done
-        ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (j - 1) & 1, abort_flag, p.err));
-        if (!ok) break;
-        tc_fence_after();
-      }
-      if (__any_sync(0xffffffffu, move)) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_off + 256 + c * 32, r);
+      if (__any_sync(0xffffffffu, move)) {  // O_t is stable: PV_t(j-1) completed before S_t(j)
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          uint32_t r[16];
+          tmem_ld16(tO + c * 16, r);
           tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-          tmem_st32(tmem + lane_off + 256 + c * 32, r);
+          for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+          tmem_st16(tO + c * 16, r);
         }
-        tmem_st_wait();
       }
-      // P row -> smem, K-major with the 128-byte swizzle: 16-byte chunk ch of row r
-      // sits at r*128 + ((ch ^ (r & 7)) * 16) inside its 64-column half.
+      // P = exp2(s * scale - m_ref), packed bf16 pairs over the first 64 columns of S_t
+      float part = 0.f;
 #pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
-        const int half = ch >> 3, cw = ch & 7;
-        uint8_t* dst = sP + half * HALF + row * 128 + ((cw ^ (row & 7)) << 4);
-        *reinterpret_cast<uint4*>(dst) = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = ex2(fmaf(s[c * 32 + 2 * e], p.scale_log2, -m_ref));
+          const float p1 = ex2(fmaf(s[c * 32 + 2 * e + 1], p.scale_log2, -m_ref));
+          part += p0 + p1;
+          pk[e] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tS + c * 16, pk);
       }
-      fence_proxy_async_smem();
+      l_sum += part;
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[t]);
     }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (n_kv - 1) & 1, abort_flag, p.err));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_full[t], 0, abort_flag, p.err));
     if (ok) {
       tc_fence_after();
-      const int qrow = qt * TILE + row;
+      const int qrow = pair * 2 * TILE + t * TILE + row;
       const float inv = 1.0f / l_sum;
       __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) + (size_t)(seg0 + qrow) * p.ldo + col0;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t r[32];
         __syncwarp();
-        tmem_ld32(tmem + lane_off + 256 + c * 32, r);
+        tmem_ld32(tO + c * 32, r);
         tmem_ld_wait();
         if (qrow < L) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
@@ -304,7 +310,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   }
   __syncthreads();
-  if (warp == 1) {
+  if (warp == WARP_MMA) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -318,11 +324,11 @@ zdit_status launch_attention(const AttnArgs& a, cudaStream_t s) {
   if ((reinterpret_cast<uintptr_t>(a.q) | reinterpret_cast<uintptr_t>(a.k) | reinterpret_cast<uintptr_t>(a.v) |
        reinterpret_cast<uintptr_t>(a.o)) & 15)
     return ZDIT_ERR_ALIGNMENT;
-  int total_qt = 0;
+  int total_pairs = 0;
   for (int b = 0; b < a.batch; ++b) {
     const int L = a.cu_seqlens_host[b + 1] - a.cu_seqlens_host[b];
     if (L <= 0) return ZDIT_ERR_SHAPE;
-    total_qt += (L + TILE - 1) / TILE;
+    total_pairs += ((L + TILE - 1) / TILE + 1) / 2;
   }
   if (a.cu_seqlens_host[0] != 0 || a.cu_seqlens_host[a.batch] > a.T) return ZDIT_ERR_SHAPE;
   CUtensorMap tq, tk, tv;
@@ -350,7 +356,7 @@ zdit_status launch_attention(const AttnArgs& a, cudaStream_t s) {
     l2 += L * L;
   }
   ProfScope ps(PROF_ATTENTION, 4.0 * HD * a.n_heads * l2, 4.0 * 2.0 * a.T * (double)cols, s);
-  dim3 grid(total_qt, a.n_heads);
+  dim3 grid(total_pairs, a.n_heads);
   attn_tc_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? ZDIT_OK : ZDIT_ERR_CUDA;
 }
