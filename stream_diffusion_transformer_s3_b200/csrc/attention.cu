@@ -240,9 +240,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int e = 0; e < TILE; ++e)
           if (e >= valid) s[e] = -INFINITY;
       }
-      float mx = -INFINITY;
+      // row max as 8 independent chains (a single 128-long chain is latency-bound)
+      float m8[8];
 #pragma unroll
-      for (int e = 0; e < TILE; ++e) mx = fmaxf(mx, s[e]);
+      for (int i = 0; i < 8; ++i) m8[i] = s[i];
+#pragma unroll
+      for (int e = 8; e < TILE; e += 8)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], s[e + i]);
+      float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                       fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       mx *= p.scale_log2;
       float alpha = 1.f;
       bool move = false;
@@ -266,7 +273,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       // P = exp2(s * scale - m_ref), packed bf16 pairs over the first 64 columns of S_t
-      float part = 0.f;
+      float part[4] = {0.f, 0.f, 0.f, 0.f};  // 4 independent sum chains
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
@@ -274,12 +281,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int e = 0; e < 16; ++e) {
           const float p0 = ex2(fmaf(s[c * 32 + 2 * e], p.scale_log2, -m_ref));
           const float p1 = ex2(fmaf(s[c * 32 + 2 * e + 1], p.scale_log2, -m_ref));
-          part += p0 + p1;
+          part[e & 3] += p0 + p1;
           pk[e] = pack_bf16x2(p0, p1);
         }
         tmem_st16(tS + c * 16, pk);
       }
-      l_sum += part;
+      l_sum += (part[0] + part[1]) + (part[2] + part[3]);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();

@@ -21,6 +21,7 @@
 #include <cudaTypedefs.h>
 
 #include <cstdio>
+#include <cstdlib>
 #include <mutex>
 
 #include "internal.h"
@@ -48,11 +49,19 @@ struct KParams {
   const float* kn;
   float eps;
   int dim;
-  int num_m, num_n, num_k, group_m;
+  int num_m, num_n, num_k, group_m, raster;
   int* err;
 };
 
+// Tile order of the persistent loop.  raster 0: M fastest inside bands of group_m
+// M-tiles; raster 1: N fastest.  The host picks the order that keeps the smaller
+// operand resident in L2 while the larger one streams from HBM once.
 __device__ __forceinline__ void tile_coords(int t, const KParams& p, int& mb, int& nb) {
+  if (p.raster == 1) {
+    mb = t / p.num_n;
+    nb = t - mb * p.num_n;
+    return;
+  }
   const int group = p.group_m * p.num_n;
   const int g = t / group;
   const int first = g * p.group_m;
@@ -311,6 +320,168 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
+// ------------------------------------------------------------------------------
+// CTA-pair variant (cta_group::2): a cluster of two CTAs computes a 256 x 256 tile.
+// Each CTA TMA-loads its own 128 rows of A and its own 128 rows of B per 64-deep
+// k-slice (32 KB per stage, 6 stages) and counts the bytes on the leader's barrier;
+// the leader's single MMA thread issues M=256 x N=256 MMAs that read both CTAs'
+// shared memory and write 128 rows x 256 columns into each CTA's TMEM; commits are
+// multicast to both CTAs.  Each CTA runs the same epilogue on its 128 rows.  Per
+// SM this halves the B traffic and gives the ring 50% more stages than the single
+// CTA kernel.  No TMA multicast is used.
+constexpr int P_STAGES = 6;
+constexpr int P_A_TILE = 128 * BK * 2;  // 16 KB
+constexpr int P_B_TILE = 128 * BK * 2;  // 16 KB
+constexpr int P_STAGE_BYTES = P_A_TILE + P_B_TILE;
+constexpr int P_SMEM_BYTES = 1024 + P_STAGES * P_STAGE_BYTES + 256;
+
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const KParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + P_STAGES * P_STAGE_BYTES);
+  uint64_t* empty = full + P_STAGES;
+  uint64_t* tfull = empty + P_STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* done = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+  const int n_pairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 8);  // 4 epilogue warps in each CTA of the pair
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) tmem_alloc_pair(tmem_slot, TMEM_COLS);
+  tc_fence_before();
+  cluster_sync();  // barriers of both CTAs initialised before any cross-CTA traffic
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int num_tiles = p.num_m * p.num_n;  // num_m counts 256-row pair tiles
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t armed = 0, armed_par = 0;
+    for (int t = pair; t < num_tiles && !*abort_flag; t += n_pairs) {
+      int mb, nb;
+      tile_coords(t, p, mb, nb);
+      const int m0 = mb * 256 + (int)rank * 128;
+      const int n0 = nb * BN + (int)rank * 128;
+      for (int kb = 0; kb < p.num_k; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err)) break;
+        uint8_t* sa = smem + stage * P_STAGE_BYTES;
+        if (leader) mbar_arrive_expect_tx(&full[stage], 2 * P_STAGE_BYTES);
+        const uint32_t bar = leader_smem_addr(&full[stage]);
+        tma_load_2d_pair(sa, &tmA, bar, kb * BK, m0);
+        tma_load_2d_pair(sa + P_A_TILE, &tmB, bar, kb * BK, n0);
+        armed |= 1u << stage;
+        armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+        if (++stage == P_STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    if (*abort_flag && leader) {
+      // the leader's full barriers also count the peer's bytes: drain both CTAs' copies
+      int dummy = 0;
+      for (int s = 0; s < P_STAGES; ++s)
+        if (armed & (1u << s)) mbar_wait(&full[s], (armed_par >> s) & 1u, &dummy);
+    }
+  } else if (warp == 1 && lane == 0 && leader) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    const uint32_t idesc = idesc_bf16_f32(256, BN);
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = pair; t < num_tiles && !*abort_flag; t += n_pairs) {
+      if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.err)) break;
+      tc_fence_after();
+      const uint32_t d = tmem_base + acc * BN;
+      bool ok = true;
+      for (int kb = 0; kb < p.num_k; ++kb) {
+        if (!mbar_wait(&full[stage], phase, abort_flag, p.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(smem + stage * P_STAGE_BYTES);
+        const uint32_t b0 = a0 + P_A_TILE;
+#pragma unroll
+        for (int k = 0; k < BK / 16; ++k)
+          umma_pair_bf16_ss(d, sdesc_kmajor_sw128(a0 + k * 32), sdesc_kmajor_sw128(b0 + k * 32), idesc,
+                            (kb | k) != 0 ? 1u : 0u);
+        umma_pair_commit_mc(&empty[stage], 0x3);
+        if (++stage == P_STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (!ok) break;
+      umma_pair_commit_mc(&tfull[acc], 0x3);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1;
+    }
+    umma_pair_commit(done);
+    int dummy = 0;
+    mbar_wait(done, 0, &dummy);
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int lg = warp & 3;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = pair; t < num_tiles; t += n_pairs) {
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err));
+      if (!ok) break;
+      tc_fence_after();
+      int mb, nb;
+      tile_coords(t, p, mb, nb);
+      const uint32_t taddr = tmem_base + ((uint32_t)(lg * 32) << 16) + acc * BN;
+      epilogue_tile<EPI>(p, taddr, mb * 256 + (int)rank * 128 + lg * 32 + lane, nb);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader)
+          mbar_arrive(&tempty[acc]);
+        else
+          mbar_arrive_cluster(&tempty[acc], 0);
+      }
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1;
+    }
+  }
+  tc_fence_before();
+  cluster_sync();  // no CTA leaves while its pair may still touch its shared memory
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -325,16 +496,26 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 template <int EPI>
-zdit_status launch_epi(const CUtensorMap& ta, const CUtensorMap& tb, const KParams& kp, int grid,
+zdit_status launch_epi(const CUtensorMap& ta, const CUtensorMap& tb, const KParams& kp, int grid, bool pair,
                        cudaStream_t s) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(gemm_tc_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
-        cudaSuccess)
-      return ZDIT_ERR_CUDA;
-    attr_set = true;
+  static bool attr_set = false, attr_pair_set = false;
+  if (pair) {
+    if (!attr_pair_set) {
+      if (cudaFuncSetAttribute(gemm_pair_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_BYTES) !=
+          cudaSuccess)
+        return ZDIT_ERR_CUDA;
+      attr_pair_set = true;
+    }
+    gemm_pair_kernel<EPI><<<grid, THREADS, P_SMEM_BYTES, s>>>(ta, tb, kp);
+  } else {
+    if (!attr_set) {
+      if (cudaFuncSetAttribute(gemm_tc_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
+          cudaSuccess)
+        return ZDIT_ERR_CUDA;
+      attr_set = true;
+    }
+    gemm_tc_kernel<EPI><<<grid, THREADS, SMEM_BYTES, s>>>(ta, tb, kp);
   }
-  gemm_tc_kernel<EPI><<<grid, THREADS, SMEM_BYTES, s>>>(ta, tb, kp);
   return cudaGetLastError() == cudaSuccess ? ZDIT_OK : ZDIT_ERR_CUDA;
 }
 
@@ -354,6 +535,17 @@ bool make_tmap_bf16_2d(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t 
   return r == CUDA_SUCCESS;
 }
 
+// ZDIT_GEMM_SINGLE_CTA=1 in the environment selects the single-CTA kernel for every
+// shape (A/B comparisons of the two kernels).
+bool force_single_cta() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("ZDIT_GEMM_SINGLE_CTA");
+    v = (e != nullptr && e[0] == '1') ? 1 : 0;
+  }
+  return v == 1;
+}
+
 zdit_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
   if (a.M <= 0 || a.N <= 0 || a.K <= 0) return ZDIT_ERR_SHAPE;
   if (a.K % 8 || a.lda % 8 || a.ldb % 8 || a.N % 32) return ZDIT_ERR_SHAPE;
@@ -364,28 +556,40 @@ zdit_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
   if (a.epi == EPI_QKV && (a.N != 3 * a.dim || a.dim % 128 || a.N % BN || !a.rope_cos || !a.rope_sin))
     return ZDIT_ERR_SHAPE;
   if ((a.epi == EPI_F32 || a.epi == EPI_BF16) && (a.ldo % 4)) return ZDIT_ERR_ALIGNMENT;
+  // CTA pairs for every shape that fills several 256 x 256 tiles; the single-CTA
+  // kernel for small or narrow problems (embedders, final layer, tiny blocks).
+  const bool pair = a.M > 256 && a.N % BN == 0 && !force_single_cta();
   CUtensorMap ta, tb;
   if (!make_tmap_bf16_2d(&ta, a.A, a.M, a.K, a.lda, BM, BK)) return ZDIT_ERR_CUDA;
-  if (!make_tmap_bf16_2d(&tb, a.B, a.N, a.K, a.ldb, BN, BK)) return ZDIT_ERR_CUDA;
+  if (!make_tmap_bf16_2d(&tb, a.B, a.N, a.K, a.ldb, pair ? 128 : BN, BK)) return ZDIT_ERR_CUDA;
   KParams kp;
   kp.M = a.M; kp.N = a.N; kp.K = a.K; kp.ldo = a.ldo; kp.out = a.out; kp.bias = a.bias;
   kp.rcos = a.rope_cos; kp.rsin = a.rope_sin; kp.qn = a.qn; kp.kn = a.kn; kp.eps = a.eps; kp.dim = a.dim;
-  kp.num_m = (a.M + BM - 1) / BM;
+  kp.num_m = pair ? (a.M + 255) / 256 : (a.M + BM - 1) / BM;
   kp.num_n = (a.N + BN - 1) / BN;
   kp.num_k = (a.K + BK - 1) / BK;
-  kp.group_m = 16;
+  // Whichever operand is smaller stays L2-resident: with A (activations) smaller,
+  // sweep every M tile of an N column before moving on (B read from HBM once, A
+  // re-read from L2); otherwise sweep N fastest (A read once, B re-read from L2).
+  const double a_bytes = 2.0 * a.M * a.K, b_bytes = 2.0 * a.N * a.K;
+  kp.raster = a_bytes <= b_bytes ? 0 : 1;
+  kp.group_m = kp.num_m;
   kp.err = device_error_ptr();
   const int tiles = kp.num_m * kp.num_n;
+  int grid = tiles < num_sms() ? tiles : num_sms();
+  if (pair) {
+    const int pairs = num_sms() / 2;
+    grid = 2 * (tiles < pairs ? tiles : pairs);
+  }
   const double out_elt = (a.epi == EPI_F32) ? 4.0 : 2.0;
   const double out_cols = (a.epi == EPI_SWIGLU) ? a.N / 2.0 : (double)a.N;
   ProfScope ps(a.prof_kind, 2.0 * a.M * a.N * (double)a.K,
                2.0 * ((double)a.M * a.K + (double)a.N * a.K) + out_elt * a.M * out_cols, s);
-  const int grid = tiles < num_sms() ? tiles : num_sms();
   switch (a.epi) {
-    case EPI_F32: return launch_epi<EPI_F32>(ta, tb, kp, grid, s);
-    case EPI_BF16: return launch_epi<EPI_BF16>(ta, tb, kp, grid, s);
-    case EPI_QKV: return launch_epi<EPI_QKV>(ta, tb, kp, grid, s);
-    case EPI_SWIGLU: return launch_epi<EPI_SWIGLU>(ta, tb, kp, grid, s);
+    case EPI_F32: return launch_epi<EPI_F32>(ta, tb, kp, grid, pair, s);
+    case EPI_BF16: return launch_epi<EPI_BF16>(ta, tb, kp, grid, pair, s);
+    case EPI_QKV: return launch_epi<EPI_QKV>(ta, tb, kp, grid, pair, s);
+    case EPI_SWIGLU: return launch_epi<EPI_SWIGLU>(ta, tb, kp, grid, pair, s);
   }
   return ZDIT_ERR_INVALID_ARG;
 }
