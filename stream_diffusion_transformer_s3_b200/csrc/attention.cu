@@ -47,6 +47,9 @@ constexpr int OFF_V = OFF_K + 2 * TILE_BYTES;
 constexpr int OFF_BAR = OFF_V + 2 * TILE_BYTES;
 constexpr int SMEM_BYTES = 1024 + OFF_BAR + 256;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Of every 4 pairs of exponentials, how many run on the FMA pipe (exp2_poly2)
+// instead of MUFU.  Measured on B200: MUFU is not the limit of this kernel, so 0.
+constexpr int kPolyPairsPer4 = 0;
 
 struct AParams {
   int ldo, n_heads, batch;
@@ -60,6 +63,57 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Packed pairs of fp32 (Blackwell f32x2 arithmetic: one instruction, two lanes).
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpk2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// 2^x for a pair, on the FMA/ALU pipes instead of MUFU, for x <= 8 (x may be -inf).
+// x is clamped to -125 (below that the result is 0), split as x = n + f with n = round(x) (the 1.5 * 2^23 shift
+// trick) and f in [-1/2, 1/2]; 2^f is a cubic fitted in relative error on that
+// interval by least squares (max relative error 2.2e-4, far below the bf16
+// rounding of P); 2^n is added into the exponent field.
+__device__ __forceinline__ void exp2_poly2(uint64_t x2, float& y0, float& y1) {
+  float a0, b0;
+  unpk2(x2, a0, b0);
+  const float a = fmaxf(a0, -125.f), b = fmaxf(b0, -125.f);  // keeps 2^n a normal number
+  const uint64_t shift = pk2(12582912.0f, 12582912.0f);
+  const uint64_t nshift = pk2(-12582912.0f, -12582912.0f);
+  const uint64_t xc = pk2(a, b);
+  const uint64_t t = add2(xc, shift);              // round(x) in the low mantissa bits
+  const uint64_t f = add2(xc, add2(t, nshift) ^ 0x8000000080000000ull);  // x - round(x)
+  uint64_t q = pk2(5.286743492e-02f, 5.286743492e-02f);
+  q = fma2(q, f, pk2(2.421518862e-01f, 2.421518862e-01f));
+  q = fma2(q, f, pk2(6.935867667e-01f, 6.935867667e-01f));
+  q = fma2(q, f, pk2(9.999627471e-01f, 9.999627471e-01f));
+  float q0, q1, t0, t1;
+  unpk2(q, q0, q1);
+  unpk2(t, t0, t1);
+  y0 = a0 < -125.f ? 0.f : __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  y1 = b0 < -125.f ? 0.f : __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 
 __global__ void __launch_bounds__(THREADS, 1)
@@ -240,16 +294,15 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int e = 0; e < TILE; ++e)
           if (e >= valid) s[e] = -INFINITY;
       }
-      // row max as 8 independent chains (a single 128-long chain is latency-bound)
+      // row max: 8 independent chains of 3-input max (a single chain is latency-bound)
       float m8[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) m8[i] = s[i];
+      for (int i = 0; i < 8; ++i) m8[i] = fmaxf(s[i], s[8 + i]);
 #pragma unroll
-      for (int e = 8; e < TILE; e += 8)
+      for (int e = 16; e < TILE; e += 16)
 #pragma unroll
-        for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], s[e + i]);
-      float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                       fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        for (int i = 0; i < 8; ++i) m8[i] = fmax3(m8[i], s[e + i], s[e + 8 + i]);
+      float mx = fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], fmax3(m8[5], m8[6], m8[7])));
       mx *= p.scale_log2;
       float alpha = 1.f;
       bool move = false;
@@ -273,20 +326,37 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       // P = exp2(s * scale - m_ref), packed bf16 pairs over the first 64 columns of S_t
-      float part[4] = {0.f, 0.f, 0.f, 0.f};  // 4 independent sum chains
+      // P = exp2(s * scale - m_ref) with packed f32x2 arithmetic (optionally a share
+      // of the exponentials on the FMA pipe, kPolyPairsPer4).
+      const uint64_t sc2 = pk2(p.scale_log2, p.scale_log2);
+      const uint64_t nm2 = pk2(-m_ref, -m_ref);
+      uint64_t part[4] = {0ull, 0ull, 0ull, 0ull};  // 4 independent packed sum chains
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float p0 = ex2(fmaf(s[c * 32 + 2 * e], p.scale_log2, -m_ref));
-          const float p1 = ex2(fmaf(s[c * 32 + 2 * e + 1], p.scale_log2, -m_ref));
-          part[e & 3] += p0 + p1;
+          const uint64_t x2 = fma2(pk2(s[c * 32 + 2 * e], s[c * 32 + 2 * e + 1]), sc2, nm2);
+          float p0, p1;
+          if ((e & 3) >= 4 - kPolyPairsPer4) {
+            exp2_poly2(x2, p0, p1);
+          } else {
+            float a, b;
+            unpk2(x2, a, b);
+            p0 = ex2(a);
+            p1 = ex2(b);
+          }
+          part[e & 3] = add2(part[e & 3], pk2(p0, p1));
           pk[e] = pack_bf16x2(p0, p1);
         }
         tmem_st16(tS + c * 16, pk);
       }
-      l_sum += (part[0] + part[1]) + (part[2] + part[3]);
+      float q0, q1, q2, q3, q4, q5, q6, q7;
+      unpk2(part[0], q0, q1);
+      unpk2(part[1], q2, q3);
+      unpk2(part[2], q4, q5);
+      unpk2(part[3], q6, q7);
+      l_sum += ((q0 + q1) + (q2 + q3)) + ((q4 + q5) + (q6 + q7));
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
