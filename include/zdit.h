@@ -333,6 +333,14 @@ ZDIT_API int64_t zdit_launch_count(void);
  * ZDIT_ERR_CUDA if the stream reports a CUDA error, else ZDIT_OK. */
 ZDIT_API zdit_status zdit_device_status(void* stream);
 
+/* Health check of the bounded waits used by every pipelined kernel: launches one
+ * kernel that waits on a barrier nothing arrives on; after the library's wait limit
+ * (2 s) it gives up, latches ZDIT_ERR_DEVICE_TIMEOUT (read with
+ * zdit_device_status) and writes 2 to *result_dev (device int32; 1 would mean the
+ * wait wrongly succeeded).  The context stays usable.  Not part of the DiT path.
+ * Errors: ZDIT_ERR_INVALID_ARG, ZDIT_ERR_CUDA. */
+ZDIT_API zdit_status zdit_selftest_wait_timeout(int32_t* result_dev, void* stream);
+
 /* Static string naming a status code. */
 ZDIT_API const char* zdit_status_string(zdit_status s);
 

@@ -99,6 +99,7 @@ _SIGS = {
     "zdit_patchify": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int32, C.c_int32, C.c_int32, C.c_void_p]),
     "zdit_unpatchify": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int32, C.c_int32, C.c_int32, C.c_void_p]),
     "zdit_device_status": (C.c_int, [C.c_void_p]),
+    "zdit_selftest_wait_timeout": (C.c_int, [C.c_void_p, C.c_void_p]),
 }
 
 
@@ -273,6 +274,10 @@ def zdit_patchify(latent, tokens, stream=None):
 def zdit_unpatchify(tokens, latent, stream=None):
     Cc, H2, W2 = latent.shape
     _check(lib().zdit_unpatchify(_ptr(tokens), _ptr(latent), Cc, H2, W2, _stream(stream)), "zdit_unpatchify")
+
+
+def zdit_selftest_wait_timeout(result_dev, stream=None):
+    _check(lib().zdit_selftest_wait_timeout(_ptr(result_dev), _stream(stream)), "zdit_selftest_wait_timeout")
 
 
 def zdit_device_status(stream=None):

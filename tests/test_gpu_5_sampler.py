@@ -1,0 +1,51 @@
+"""The 8-step FlowMatchEuler sampler with negated CFG driven through the public
+calls (zdit_stack_forward on the cond/uncond pair, zdit_euler_cfg_step), at reduced
+width so the oracle's float64 sampler finishes in seconds: latent 16 x 16 x 16
+(8 x 8 patch grid), g = 1, endpoint-preserving 9-point schedule, no call at
+sigma = 0."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import stream_diffusion_transformer_s3_b200 as Z
+from stream_diffusion_transformer_s3_b200 import synth
+from _gpu import dev, dims_of, errors, host, require_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _gpu():
+    require_gpu()
+
+
+def test_eight_step_sampler_matches_oracle():
+    d = synth.BlockDims(dim=256, n_heads=2, head_dim=128, ffn_hidden=384)
+    W = synth.stack_weights(9, d, n_noise=2, n_context=2, n_main=2, cap_dim=128)
+    latent = synth.latent_noise(42, (16, 16, 16))
+    caps = synth.randn(9, 300, (46, 128))
+    cond = {"caps": caps[:45], "n_cap": 64, "n_valid": 45}
+    unc = {"caps": caps[45:], "n_cap": 32, "n_valid": 1}
+
+    stack = Z.DeviceStack(W, dims_of(d), 2, 2, 2, patch_dim=64, cap_dim=128)
+    z = torch.empty(64, 64, device="cuda")
+    Z.zdit_patchify(dev(latent), z)
+    call = Z.StackCall((8, 8), [64, 32], [45, 1], [0.0, 0.0], z, dev(caps), shared_patches=True)
+    ws = torch.empty(Z.stack_workspace_bytes(stack, call), dtype=torch.uint8, device="cuda")
+    out = torch.empty(2, 64, 64, device="cuda")
+    sig = Z.zdit_sigma_schedule(8)
+    calls = 0
+    for i in range(8):
+        call.set_t([1.0 - sig[i]] * 2)
+        Z.zdit_stack_forward(stack, call, out, ws)
+        calls += 1
+        Z.zdit_euler_cfg_step(z, out[0], out[1], 1.0, sig[i], sig[i + 1])
+    assert sig[8] == 0.0 and calls == 8
+    result = torch.empty(16, 16, 16, device="cuda")
+    Z.zdit_unpatchify(z, result)
+    assert Z.zdit_device_status() == 0
+    ref = O.sample(latent, cond, unc, W, d, g=1.0, n_steps=8)
+    e = errors(host(result), ref)
+    print("\nsampler", e)
+    assert e["rel_l2"] <= 2e-2, e
