@@ -169,8 +169,8 @@ ZDIT_API zdit_status zdit_block_forward(const zdit_block_cfg* cfg, const zdit_bl
  *   workspace is a 40 MiB device array owned by the library (held on every GPU that
  *   loads the library until the process exits); calls needing more than 40 MiB of
  *   workspace (zdit_block_workspace_bytes) return ZDIT_ERR_WORKSPACE and launch
- *   nothing.  At full width (D 3840, F 10240, two branches) that admits up to 777 tokens,
- *   e.g. the 256px cond/uncond pair (608 tokens).
+ *   nothing.  At full width (D 3840, F 10240, two branches) that admits up to 907 tokens,
+ *   e.g. the 256px cond/uncond pair (608 tokens, 26.8 MiB).
  *   The call allocates nothing (no cudaMalloc, cudaFree or allocating library call).
  *   The first call on a device looks up the array's device address (once per
  *   device, with that device current); make that first call before any stream

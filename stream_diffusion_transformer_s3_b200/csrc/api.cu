@@ -93,7 +93,7 @@ struct BlockWs {
   __nv_bfloat16* a;     // [T, D]
   __nv_bfloat16* qkvh;  // [T, max(3D, F)]
   __nv_bfloat16* o;     // [T, D]
-  float* y;             // [T, D]
+  __nv_bfloat16* y;     // [T, D] projection output before the sandwich norm
 };
 
 size_t carve_block(Carver& c, BlockWs* ws, int64_t T, int B, int D, int F) {
@@ -103,7 +103,7 @@ size_t carve_block(Carver& c, BlockWs* ws, int64_t T, int B, int D, int F) {
   w.a = c.take<__nv_bfloat16>((size_t)T * D);
   w.qkvh = c.take<__nv_bfloat16>((size_t)T * wide);
   w.o = c.take<__nv_bfloat16>((size_t)T * D);
-  w.y = c.take<float>((size_t)T * D);
+  w.y = c.take<__nv_bfloat16>((size_t)T * D);
   if (ws) *ws = w;
   return c.off;
 }
@@ -119,11 +119,19 @@ bool varlen_ok(const zdit_varlen* v) {
 
 inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
+// Next block's pre-attention norm, fused into this block's last residual kernel.
+struct NextNorm {
+  const float* w;      // next block's n_attn
+  const float* scale;  // next block's scale_attn [B, 4D] base (nullptr without adaLN)
+};
+
 // The block's launch sequence.  `mod` holds the adaLN vectors [B, 4D] (ignored
-// without ADALN).
+// without ADALN).  a_ready: ws.a already holds this block's pre-attention operand
+// (written by the previous block's fused residual); next: fuse the next block's
+// pre-attention norm into the final residual kernel.
 zdit_status run_block(const zdit_block_cfg& cfg, const zdit_block_weights& w, const zdit_varlen& vl, int T,
                       float* x, const float* mod, const float* rcos, const float* rsin, const BlockWs& ws,
-                      cudaStream_t s) {
+                      cudaStream_t s, bool a_ready = false, const NextNorm* next = nullptr) {
   const int D = cfg.dim, F = cfg.ffn_hidden, B = vl.batch;
   const bool adaln = cfg.flags & ZDIT_F_ADALN;
   const bool sandwich = cfg.flags & ZDIT_F_SANDWICH_NORM;
@@ -135,7 +143,8 @@ zdit_status run_block(const zdit_block_cfg& cfg, const zdit_block_weights& w, co
   const int ms = 4 * D;
 
   // pre-attention norm + modulation -> bf16 operand
-  launch_norm_modulate_ex(x, T, D, w.n_attn, s1, ms, vl.cu_seqlens_dev, B, 0, 0, cfg.norm_eps, ws.a, s);
+  if (!a_ready)
+    launch_norm_modulate_ex(x, T, D, w.n_attn, s1, ms, vl.cu_seqlens_dev, B, 0, 0, cfg.norm_eps, ws.a, s);
 
   // QKV projection with (QK-norm +) RoPE epilogue -> [T, 3D] bf16
   GemmArgs g{};
@@ -157,7 +166,7 @@ zdit_status run_block(const zdit_block_cfg& cfg, const zdit_block_weights& w, co
   // output projection -> y fp32
   GemmArgs go{};
   go.A = ws.o; go.lda = D; go.B = w.w_out; go.ldb = D; go.M = T; go.N = D; go.K = D;
-  go.epi = EPI_F32; go.out = ws.y; go.ldo = D; go.prof_kind = PROF_GEMM_OUT;
+  go.epi = EPI_BF16; go.out = ws.y; go.ldo = D; go.prof_kind = PROF_GEMM_OUT;
   st = launch_gemm(go, s);
   if (st != ZDIT_OK) return st;
 
@@ -179,7 +188,7 @@ zdit_status run_block(const zdit_block_cfg& cfg, const zdit_block_weights& w, co
   // down projection -> y fp32
   GemmArgs gd{};
   gd.A = ws.qkvh; gd.lda = F; gd.B = w.w_down; gd.ldb = F; gd.M = T; gd.N = D; gd.K = F;
-  gd.epi = EPI_F32; gd.out = ws.y; gd.ldo = D; gd.prof_kind = PROF_GEMM_DOWN;
+  gd.epi = EPI_BF16; gd.out = ws.y; gd.ldo = D; gd.prof_kind = PROF_GEMM_DOWN;
   st = launch_gemm(gd, s);
   if (st != ZDIT_OK) return st;
 
@@ -187,7 +196,11 @@ zdit_status run_block(const zdit_block_cfg& cfg, const zdit_block_weights& w, co
   ResidArgs r2 = r;
   r2.post_w = sandwich ? w.n_ffn_post : nullptr;
   r2.gate = g2;
-  r2.next_w = nullptr; r2.next_scale = nullptr; r2.next_out = nullptr;
+  if (next != nullptr) {
+    r2.next_w = next->w; r2.next_scale = next->scale; r2.next_out = ws.a;
+  } else {
+    r2.next_w = nullptr; r2.next_scale = nullptr; r2.next_out = nullptr;
+  }
   launch_residual(r2, s);
   return cudaGetLastError() == cudaSuccess ? ZDIT_OK : ZDIT_ERR_CUDA;
 }
@@ -451,10 +464,19 @@ ZDIT_API zdit_status zdit_stack_forward(const zdit_stack_cfg* cfg, const zdit_st
                         (size_t)d.n_cap[b] * D * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
       return ZDIT_ERR_CUDA;
   }
-  // main blocks
-  for (int i = cfg->n_noise_refiner + cfg->n_context_refiner; i < d.nblk; ++i) {
+  // main blocks; each one's last residual kernel also produces the next block's
+  // pre-attention operand
+  const int first_main = cfg->n_noise_refiner + cfg->n_context_refiner;
+  const bool adaln = bcfg.flags & ZDIT_F_ADALN;
+  for (int i = first_main; i < d.nblk; ++i) {
+    NextNorm nn{};
+    const bool has_next = i + 1 < d.nblk;
+    if (has_next) {
+      nn.w = w->blocks[i + 1].n_attn;
+      nn.scale = adaln ? ws.mods + (size_t)(i + 1) * B * 4 * D : nullptr;
+    }
     st = run_block(bcfg, w->blocks[i], v_joint, d.T, ws.x_joint, ws.mods + (size_t)i * B * 4 * D, ws.cos_joint,
-                   ws.sin_joint, ws.blk, s);
+                   ws.sin_joint, ws.blk, s, i > first_main, has_next ? &nn : nullptr);
     if (st != ZDIT_OK) return st;
   }
   // final layer on the image rows of each branch

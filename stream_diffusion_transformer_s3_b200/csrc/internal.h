@@ -93,7 +93,7 @@ void launch_norm_modulate(const RowModArgs& a, cudaStream_t s);
 
 struct ResidArgs {
   float* x;              // [T, D] in/out residual stream
-  const float* y;        // [T, D] projection output
+  const __nv_bfloat16* y;  // [T, D] projection output (bf16)
   int T, D;
   const float* post_w;   // sandwich norm weight or nullptr (no post-norm)
   const float* gate;     // per-branch gate: gate[b*gate_stride + d], or nullptr (gate 1)

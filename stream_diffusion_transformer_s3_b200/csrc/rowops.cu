@@ -3,8 +3,8 @@
 //   norm_modulate : a = Norm(x) * w * (1 + scale_b) -> bf16 GEMM operand
 //                   (RMSNorm pre-norm of the block; LayerNorm without affine for the
 //                   final layer; plain RMSNorm for the caption embedder)
-//   residual      : x += gate_b * PostNorm(y), optionally fused with the next
-//                   pre-norm so x is read once per step
+//   residual      : x += gate_b * PostNorm(y) (y bf16), optionally fused with the
+//                   next pre-norm so x is read once per step
 //   adaln_gemv    : m_b = W_ada temb_b + b_ada (weight-streaming GEMV)
 //   euler_cfg     : x += (sigma_next - sigma_cur) * -(pos + g (pos - neg))
 //   rope_table    : per-token cos/sin of the 3-axis rotary angles
@@ -142,7 +142,7 @@ __global__ void __launch_bounds__(RT) norm_modulate_kernel(NormModParams p) {
 
 struct ResidParams {
   float* x;
-  const float* y;
+  const __nv_bfloat16* y;
   int D;
   const float* post_w;
   const float* gate;
@@ -161,14 +161,21 @@ template <int MAXV>
 __global__ void __launch_bounds__(RT) residual_kernel(ResidParams p) {
   __shared__ float sh[RT / 32];
   const int t = blockIdx.x;
-  const float* yr = p.y + (size_t)t * p.D;
+  const __nv_bfloat16* yr = p.y + (size_t)t * p.D;
   float* xr = p.x + (size_t)t * p.D;
   float4 y[MAXV];
   float ss = 0.f;
 #pragma unroll
   for (int i = 0; i < MAXV; ++i) {
     const int idx = (i * RT + threadIdx.x) * 4;
-    y[i] = idx < p.D ? *reinterpret_cast<const float4*>(yr + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
+    if (idx < p.D) {
+      const uint2 u = *reinterpret_cast<const uint2*>(yr + idx);
+      const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
+      const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
+      y[i] = make_float4(__low2float(lo), __high2float(lo), __low2float(hi), __high2float(hi));
+    } else {
+      y[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     ss += y[i].x * y[i].x + y[i].y * y[i].y + y[i].z * y[i].z + y[i].w * y[i].w;
   }
   float r = 1.f;
@@ -445,7 +452,7 @@ void launch_norm_modulate(const RowModArgs& a, cudaStream_t s) {
 }
 
 void launch_residual(const ResidArgs& a, cudaStream_t s) {
-  ProfScope ps(PROF_RESIDUAL, 0.0, (double)a.T * a.D * (12.0 + (a.next_out ? 2.0 : 0.0)), s);
+  ProfScope ps(PROF_RESIDUAL, 0.0, (double)a.T * a.D * (10.0 + (a.next_out ? 2.0 : 0.0)), s);
   ResidParams p{a.x,       a.y,    a.D,          a.post_w,  a.gate,       a.gate_stride, a.tanh_gate,
                 a.cu_seqlens, a.batch, a.eps,    a.next_w,  a.next_scale, a.next_scale_stride, a.next_out};
   const int v = (a.D + RT * 4 - 1) / (RT * 4);

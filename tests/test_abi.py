@@ -49,8 +49,8 @@ def test_block_workspace_sizing():
     small = Z.block_workspace_bytes(d, f, 608, 2)
     big = Z.block_workspace_bytes(d, f, 8352, 2)
     assert 0 < small < big
-    # activations alone: a, o (bf16 D) + qkv/h (bf16 max(3D, F)) + y (fp32 D) per token
-    per_tok = 2 * 3840 * 2 + 2 * 11520 + 4 * 3840
+    # activations alone: a, o, y (bf16 D each) + qkv/h (bf16 max(3D, F)) per token
+    per_tok = 3 * 2 * 3840 + 2 * 11520
     assert big >= 8352 * per_tok
     assert Z.block_workspace_bytes(Z.Dims(head_dim=64), f, 608, 2) == 0
     assert Z.block_workspace_bytes(d, f, 0, 2) == 0

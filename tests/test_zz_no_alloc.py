@@ -26,7 +26,7 @@ def _gpu():
 
 
 def test_static_scratch_block_matches_workspace_block_twice():
-    case = synth.config2(0)  # full width, cond/uncond 320 + 288 tokens (31.3 MiB of scratch)
+    case = synth.config2(0)  # full width, cond/uncond 320 + 288 tokens (26.8 MiB of scratch)
     d = synth.FULL
     dims = dims_of(d)
     fl = Z.flags_of()
