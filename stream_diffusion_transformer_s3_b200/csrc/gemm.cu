@@ -15,8 +15,9 @@
 // FP32, bf16 storage, never fp16):
 //   EPI_F32    fp32 store (+ bias)                 out-proj, w2, embedders
 //   EPI_BF16   bf16 store (+ bias)
-//   EPI_QKV    q/k columns: optional per-head RMSNorm, then real interleaved RoPE
-//              with per-token cos/sin; bf16 store of [q | k | v]
+//   EPI_QKV    q/k columns: real interleaved RoPE with per-token cos/sin, 32-column
+//              chunks; bf16 store of [q | k | v]
+//   EPI_QKV_NORM  same with a per-head RMSNorm of q and k first (whole head at once)
 //   EPI_SWIGLU gate/up column blocks -> silu(gate) * up, bf16 store
 #include <cudaTypedefs.h>
 
@@ -133,6 +134,46 @@ __device__ __forceinline__ void epilogue_tile(const KParams& p, uint32_t taddr, 
       }
     }
   } else if constexpr (EPI == EPI_QKV) {
+    {
+      // RoPE pairs never cross a 32-column chunk, so work chunk by chunk
+      // (cos/sin of the 16 pairs of the chunk) and keep register use low.
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        const int col0 = nb * BN + c * 32;
+        uint32_t r[32];
+        __syncwarp();
+        tmem_ld32(taddr + c * 32, r);
+        tmem_ld_wait();
+        if (!row_ok) continue;
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+        if (col0 < 2 * p.dim) {  // q or k columns: rotate
+          const int pair0 = (col0 & 127) >> 1;  // first pair index of the chunk inside its head
+          const float4* cs = reinterpret_cast<const float4*>(p.rcos + (size_t)row * 64 + pair0);
+          const float4* sn = reinterpret_cast<const float4*>(p.rsin + (size_t)row * 64 + pair0);
+#pragma unroll
+          for (int i4 = 0; i4 < 4; ++i4) {
+            const float4 c4 = cs[i4], s4 = sn[i4];
+            const float cc[4] = {c4.x, c4.y, c4.z, c4.w};
+            const float ss[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int i = i4 * 4 + e;
+              const float x0 = v[2 * i], x1 = v[2 * i + 1];
+              v[2 * i] = x0 * cc[e] - x1 * ss[e];
+              v[2 * i + 1] = x0 * ss[e] + x1 * cc[e];
+            }
+          }
+        }
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.ldo + col0);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          dst[j] = make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
+                              pack_bf16x2(v[8 * j + 4], v[8 * j + 5]), pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+      }
+    }
+  } else if constexpr (EPI == EPI_QKV_NORM) {
 #pragma unroll 1
     for (int hh = 0; hh < BN / 128; ++hh) {
       const int colh = nb * BN + hh * 128;
@@ -588,7 +629,9 @@ zdit_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
   switch (a.epi) {
     case EPI_F32: return launch_epi<EPI_F32>(ta, tb, kp, grid, pair, s);
     case EPI_BF16: return launch_epi<EPI_BF16>(ta, tb, kp, grid, pair, s);
-    case EPI_QKV: return launch_epi<EPI_QKV>(ta, tb, kp, grid, pair, s);
+    case EPI_QKV:
+      return a.qn != nullptr ? launch_epi<EPI_QKV_NORM>(ta, tb, kp, grid, pair, s)
+                             : launch_epi<EPI_QKV>(ta, tb, kp, grid, pair, s);
     case EPI_SWIGLU: return launch_epi<EPI_SWIGLU>(ta, tb, kp, grid, pair, s);
   }
   return ZDIT_ERR_INVALID_ARG;

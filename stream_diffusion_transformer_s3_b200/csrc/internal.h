@@ -41,6 +41,7 @@ enum GemmEpilogue : int {
   EPI_BF16 = 1,    // out bf16 [M, ldo] = acc (+ bias[n])
   EPI_QKV = 2,     // out bf16 [M, 3D]; columns < 2D: optional per-head RMSNorm, then RoPE
   EPI_SWIGLU = 3,  // out bf16 [M, N/2]; tile columns [gate 128 | up 128] -> silu(g) * u
+  EPI_QKV_NORM = 4,  // EPI_QKV with per-head RMSNorm of q and k before RoPE (selected when qn != null)
 };
 
 struct GemmArgs {

@@ -41,22 +41,8 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
-#ifndef ZDIT_MBAR_TEST_WAIT
-#define ZDIT_MBAR_TEST_WAIT 0
-#endif
-// One poll of the barrier phase.  try_wait may park the thread for a while inside
-// the instruction; test_wait returns at once (pure spin).
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity) {
   uint32_t ok;
-#if ZDIT_MBAR_TEST_WAIT
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar_addr), "r"(parity)
-      : "memory");
-#else
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
@@ -64,7 +50,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
       : "=r"(ok)
       : "r"(bar_addr), "r"(parity)
       : "memory");
-#endif
   return ok != 0;
 }
 
