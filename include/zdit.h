@@ -253,6 +253,33 @@ ZDIT_API zdit_status zdit_stack_forward(const zdit_stack_cfg* cfg, const zdit_st
                                         const zdit_stack_inputs* in, float* out, void* workspace,
                                         size_t workspace_bytes, void* stream);
 
+/* The 8-step sampler in one call: patchify the latent, then for i < n_steps run the
+ * DiT on every branch at t = 1 - sigma_i (sigma_i = 3(1-u)/(3(1-u)+u), u = i/n_steps,
+ * ending at sigma = 0 with no call there) and apply the negated-CFG Euler update,
+ * then unpatchify ([CoreAI] Sampler row, "The three things", item 2 and "Hosting it
+ * from Swift"; [Port] sampler contract).  Branch 0 is the conditional branch, branch
+ * 1 (optional) the unconditional one; with one branch the update uses v = -pos.
+ *   cache_context: embed and refine the captions once and reuse them for every step
+ *     (the context refiner has no adaLN, so it does not depend on t).
+ *   dedup_noise: run the noise refiner once for all branches (they share the latent
+ *     and t, and their image tokens differ only in the axis-0 position, whose rotation
+ *     cancels in q.k); equal to the full computation up to rounding. */
+typedef struct {
+  int32_t n_steps;        /* sampler updates (8)                         */
+  float guidance;         /* g of -(pos + g (pos - neg)); two branches    */
+  int32_t cache_context;  /* 1: caption stream computed once             */
+  int32_t dedup_noise;    /* 1: noise refiner computed once for branches  */
+} zdit_sample_cfg;
+
+/* in: batch 1 or 2, grid, n_cap, n_valid, cap_feats as for zdit_stack_forward;
+ * patches, t and shared_patches are ignored (the sampler supplies them).
+ * latent: device fp32 [patch_dim / 4, 2 grid_h, 2 grid_w], the initial noise on
+ * entry and the final latent on return.  Errors as zdit_stack_forward. */
+ZDIT_API size_t zdit_sample_workspace_bytes(const zdit_stack_cfg* cfg, const zdit_stack_inputs* in);
+ZDIT_API zdit_status zdit_sample(const zdit_stack_cfg* cfg, const zdit_stack_weights* w,
+                                 const zdit_stack_inputs* in, const zdit_sample_cfg* sc, float* latent,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
 /* Fused negated CFG + FlowMatchEuler update over n fp32 values (device):
  *   v = -(v_pos + g * (v_pos - v_neg));  x += (sigma_next - sigma_cur) * v
  * v_neg == NULL means a single branch: v = -v_pos (g ignored).

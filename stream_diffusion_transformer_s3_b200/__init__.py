@@ -66,6 +66,11 @@ class StackInputs(C.Structure):
                 ("shared_patches", C.c_int32)]
 
 
+class SampleCfg(C.Structure):
+    _fields_ = [("n_steps", C.c_int32), ("guidance", C.c_float), ("cache_context", C.c_int32),
+                ("dedup_noise", C.c_int32)]
+
+
 class ProfileEntry(C.Structure):
     _fields_ = [("name", C.c_char * 40), ("launches", C.c_int32), ("total_ms", C.c_double),
                 ("flops", C.c_double), ("bytes", C.c_double)]
@@ -86,6 +91,9 @@ _SIGS = {
     "zdit_stack_workspace_bytes": (C.c_size_t, [C.POINTER(StackCfg), C.POINTER(StackInputs)]),
     "zdit_stack_forward": (C.c_int, [C.POINTER(StackCfg), C.POINTER(StackWeights), C.POINTER(StackInputs),
                                      C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]),
+    "zdit_sample_workspace_bytes": (C.c_size_t, [C.POINTER(StackCfg), C.POINTER(StackInputs)]),
+    "zdit_sample": (C.c_int, [C.POINTER(StackCfg), C.POINTER(StackWeights), C.POINTER(StackInputs),
+                              C.POINTER(SampleCfg), C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]),
     "zdit_euler_cfg_step": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int64, C.c_float,
                                       C.c_float, C.c_float, C.c_void_p]),
     "zdit_sigma_schedule": (C.c_int, [C.c_int32, C.POINTER(C.c_float)]),
@@ -353,3 +361,16 @@ def zdit_profile_end() -> dict:
 
 def zdit_launch_count() -> int:
     return int(lib().zdit_launch_count())
+
+
+def sample_workspace_bytes(stack: DeviceStack, call: StackCall) -> int:
+    return int(lib().zdit_sample_workspace_bytes(C.byref(stack.cfg), C.byref(call.struct)))
+
+
+def zdit_sample(stack: DeviceStack, call: StackCall, latent, workspace, n_steps=8, guidance=1.0,
+                cache_context=True, dedup_noise=False, stream=None):
+    """In-place 8-step negated-CFG FlowMatchEuler sampling of `latent` [C, 2h, 2w]."""
+    sc = SampleCfg(n_steps, guidance, 1 if cache_context else 0, 1 if dedup_noise else 0)
+    _check(lib().zdit_sample(C.byref(stack.cfg), C.byref(stack.wstruct), C.byref(call.struct), C.byref(sc),
+                             _ptr(latent), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                             _stream(stream)), "zdit_sample")

@@ -303,6 +303,123 @@ size_t carve_stack(Carver& c, StackWs* ws, const StackDims& d) {
   return c.off;
 }
 
+// The stack's launch sequence.  opts.context_ready: ws.x_cap already holds the
+// refined caption stream of these captions (the context refiner has no adaLN, so it
+// does not depend on t); opts.dedup_noise: every branch reads the same patch tokens
+// with the same t, so the noise refiner runs once on branch 0 and its result serves
+// all branches (the image tokens of a branch differ only in the axis-0 position,
+// whose rotation cancels in q.k).
+struct StackOpts {
+  bool context_ready = false;
+  bool dedup_noise = false;
+};
+
+zdit_status stack_run(const zdit_stack_cfg* cfg, const zdit_stack_weights* w, const zdit_stack_inputs* in,
+                      const StackDims& d, const StackWs& ws, float* out, const StackOpts& opts, cudaStream_t s) {
+  const int D = d.D, B = d.B, E = d.E;
+  const zdit_block_cfg& bcfg = cfg->block;
+
+  // token layout: positions and segment offsets of the three sequences
+  launch_stack_layout(d.n_cap, B, in->grid_h, in->grid_w, ws.pos_img, ws.pos_cap, ws.pos_joint, ws.cu_img,
+                      ws.cu_cap, ws.cu_joint, s);
+  launch_rope_table(ws.pos_img, d.T_img, 128, bcfg.rope_axes, bcfg.rope_theta, ws.cos_img, ws.sin_img, s);
+  launch_rope_table(ws.pos_cap, d.T_cap, 128, bcfg.rope_axes, bcfg.rope_theta, ws.cos_cap, ws.sin_cap, s);
+  launch_rope_table(ws.pos_joint, d.T, 128, bcfg.rope_axes, bcfg.rope_theta, ws.cos_joint, ws.sin_joint, s);
+
+  // timestep embedding and every adaLN vector of the forward
+  launch_timestep_embed(in->t, B, E, cfg->t_scale, static_cast<const __nv_bfloat16*>(w->w_t1), w->b_t1,
+                        static_cast<const __nv_bfloat16*>(w->w_t2), w->b_t2, ws.temb, s);
+  for (int i = 0; i < d.nblk; ++i) {
+    const bool ctx = i >= cfg->n_noise_refiner && i < cfg->n_noise_refiner + cfg->n_context_refiner;
+    if (ctx || !(bcfg.flags & ZDIT_F_ADALN)) continue;
+    launch_gemv(static_cast<const __nv_bfloat16*>(w->blocks[i].w_ada), w->blocks[i].b_ada, ws.temb, B, E, 4 * D,
+                ws.mods + (size_t)i * B * 4 * D, s);
+  }
+  launch_gemv(static_cast<const __nv_bfloat16*>(w->w_fada), w->b_fada, ws.temb, B, E, D, ws.fmod, s);
+
+  // image embedder: patches -> bf16 -> Linear(patch_dim, D) + bias
+  const int B_img = opts.dedup_noise ? 1 : B;  // branches whose image stream is computed
+  for (int b = 0; b < B_img; ++b)
+    launch_cast_bf16(in->patches + (in->shared_patches ? 0 : (size_t)b * d.n_img * d.patch_dim),
+                     ws.patches16 + (size_t)b * d.n_img * d.patch_dim, (int64_t)d.n_img * d.patch_dim, s);
+  GemmArgs gx{};
+  gx.A = ws.patches16; gx.lda = d.patch_dim; gx.B = w->w_x; gx.ldb = d.patch_dim; gx.M = B_img * d.n_img; gx.N = D;
+  gx.K = d.patch_dim; gx.epi = EPI_F32; gx.out = ws.x_img; gx.ldo = D; gx.bias = w->b_x;
+  zdit_status st = launch_gemm(gx, s);
+  if (st != ZDIT_OK) return st;
+
+  // caption embedder: RMSNorm(valid rows) -> Linear(cap_dim, D) + bias; pads <- pad_vec
+  if (!opts.context_ready) {
+  if (cudaMemsetAsync(ws.caps16, 0, (size_t)d.T_cap * d.cap_dim * sizeof(__nv_bfloat16), s) != cudaSuccess)
+    return ZDIT_ERR_CUDA;
+  for (int b = 0; b < B; ++b)
+    if (d.n_valid[b] > 0)
+      launch_norm_modulate_ex(in->cap_feats + (size_t)d.cap_off[b] * d.cap_dim, d.n_valid[b], d.cap_dim,
+                              w->w_capnorm, nullptr, 0, nullptr, 1, 0, 0, bcfg.norm_eps,
+                              ws.caps16 + (size_t)d.cu_cap[b] * d.cap_dim, s);
+  GemmArgs gc{};
+  gc.A = ws.caps16; gc.lda = d.cap_dim; gc.B = w->w_cap; gc.ldb = d.cap_dim; gc.M = d.T_cap; gc.N = D;
+  gc.K = d.cap_dim; gc.epi = EPI_F32; gc.out = ws.x_cap; gc.ldo = D; gc.bias = w->b_cap;
+  st = launch_gemm(gc, s);
+  if (st != ZDIT_OK) return st;
+  for (int b = 0; b < B; ++b)
+    launch_fill_rows(ws.x_cap + (size_t)(d.cu_cap[b] + d.n_valid[b]) * D, D, d.n_cap[b] - d.n_valid[b],
+                     w->pad_vec, s);
+  }
+
+  // refiners
+  zdit_varlen v_img{B_img, ws.cu_img, d.cu_img};
+  zdit_varlen v_cap{B, ws.cu_cap, d.cu_cap};
+  zdit_varlen v_joint{B, ws.cu_joint, d.cu_joint};
+  for (int i = 0; i < d.nblk; ++i) {
+    const bool noise = i < cfg->n_noise_refiner;
+    const bool ctx = !noise && i < cfg->n_noise_refiner + cfg->n_context_refiner;
+    if (!noise && !ctx) continue;
+    if (ctx && opts.context_ready) continue;
+    zdit_block_cfg bc = bcfg;
+    if (ctx) bc.flags &= ~ZDIT_F_ADALN;
+    const float* mod = ws.mods + (size_t)i * B * 4 * D;
+    st = noise ? run_block(bc, w->blocks[i], v_img, B_img * d.n_img, ws.x_img, mod, ws.cos_img, ws.sin_img, ws.blk, s)
+               : run_block(bc, w->blocks[i], v_cap, d.T_cap, ws.x_cap, mod, ws.cos_cap, ws.sin_cap, ws.blk, s);
+    if (st != ZDIT_OK) return st;
+  }
+  // concatenate each branch as [image | caption]
+  for (int b = 0; b < B; ++b) {
+    if (cudaMemcpyAsync(ws.x_joint + (size_t)d.cu_joint[b] * D, ws.x_img + (size_t)(opts.dedup_noise ? 0 : d.cu_img[b]) * D,
+                        (size_t)d.n_img * D * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+      return ZDIT_ERR_CUDA;
+    if (cudaMemcpyAsync(ws.x_joint + (size_t)(d.cu_joint[b] + d.n_img) * D, ws.x_cap + (size_t)d.cu_cap[b] * D,
+                        (size_t)d.n_cap[b] * D * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+      return ZDIT_ERR_CUDA;
+  }
+  // main blocks; each one's last residual kernel also produces the next block's
+  // pre-attention operand
+  const int first_main = cfg->n_noise_refiner + cfg->n_context_refiner;
+  const bool adaln = bcfg.flags & ZDIT_F_ADALN;
+  for (int i = first_main; i < d.nblk; ++i) {
+    NextNorm nn{};
+    const bool has_next = i + 1 < d.nblk;
+    if (has_next) {
+      nn.w = w->blocks[i + 1].n_attn;
+      nn.scale = adaln ? ws.mods + (size_t)(i + 1) * B * 4 * D : nullptr;
+    }
+    st = run_block(bcfg, w->blocks[i], v_joint, d.T, ws.x_joint, ws.mods + (size_t)i * B * 4 * D, ws.cos_joint,
+                   ws.sin_joint, ws.blk, s, i > first_main, has_next ? &nn : nullptr);
+    if (st != ZDIT_OK) return st;
+  }
+  // final layer on the image rows of each branch
+  for (int b = 0; b < B; ++b) {
+    launch_norm_modulate_ex(ws.x_joint + (size_t)d.cu_joint[b] * D, d.n_img, D, nullptr, ws.fmod + (size_t)b * D, 0,
+                            nullptr, 1, 0, 1, cfg->final_eps, ws.blk.a, s);
+    GemmArgs gf{};
+    gf.A = ws.blk.a; gf.lda = D; gf.B = w->w_final; gf.ldb = D; gf.M = d.n_img; gf.N = d.patch_dim; gf.K = D;
+    gf.epi = EPI_F32; gf.out = out + (size_t)b * d.n_img * d.patch_dim; gf.ldo = d.patch_dim; gf.bias = w->b_final;
+    st = launch_gemm(gf, s);
+    if (st != ZDIT_OK) return st;
+  }
+  return cudaGetLastError() == cudaSuccess ? ZDIT_OK : ZDIT_ERR_CUDA;
+}
+
 }  // namespace
 }  // namespace zdit
 
@@ -363,14 +480,13 @@ ZDIT_API size_t zdit_stack_workspace_bytes(const zdit_stack_cfg* cfg, const zdit
   return carve_stack(c, nullptr, d);
 }
 
-ZDIT_API zdit_status zdit_stack_forward(const zdit_stack_cfg* cfg, const zdit_stack_weights* w,
-                                        const zdit_stack_inputs* in, float* out, void* workspace,
-                                        size_t workspace_bytes, void* stream) {
+// Host-side checks shared by zdit_stack_forward and zdit_sample.
+zdit_status stack_validate(const zdit_stack_cfg* cfg, const zdit_stack_weights* w, const zdit_stack_inputs* in,
+                           const float* out, void* workspace, StackDims* d) {
   if (!cfg || !w || !in || !out || !workspace || !in->patches || !in->t) return ZDIT_ERR_INVALID_ARG;
-  StackDims d;
-  if (!stack_dims(cfg, in, &d)) return ZDIT_ERR_SHAPE;
-  if (d.nblk > 0 && !w->blocks) return ZDIT_ERR_INVALID_ARG;
-  if (d.cap_off[d.B] > 0 && !in->cap_feats) return ZDIT_ERR_INVALID_ARG;
+  if (!stack_dims(cfg, in, d)) return ZDIT_ERR_SHAPE;
+  if (d->nblk > 0 && !w->blocks) return ZDIT_ERR_INVALID_ARG;
+  if (d->cap_off[d->B] > 0 && !in->cap_feats) return ZDIT_ERR_INVALID_ARG;
   const void* req[] = {w->w_x, w->b_x, w->w_capnorm, w->w_cap, w->b_cap, w->pad_vec, w->w_t1, w->b_t1,
                        w->w_t2, w->b_t2, w->w_fada, w->b_fada, w->w_final, w->b_final};
   for (const void* p : req)
@@ -380,115 +496,99 @@ ZDIT_API zdit_status zdit_stack_forward(const zdit_stack_cfg* cfg, const zdit_st
   if (!al16(out) || !al16(in->patches) || (in->cap_feats && !al16(in->cap_feats)) ||
       (reinterpret_cast<uintptr_t>(workspace) & 255))
     return ZDIT_ERR_ALIGNMENT;
-  for (int i = 0; i < d.nblk; ++i) {
+  for (int i = 0; i < d->nblk; ++i) {
     zdit_block_cfg bc = cfg->block;
     if (i >= cfg->n_noise_refiner && i < cfg->n_noise_refiner + cfg->n_context_refiner) bc.flags &= ~ZDIT_F_ADALN;
     if (!block_weights_ok(bc, w->blocks[i])) return ZDIT_ERR_INVALID_ARG;
   }
   if (!device_ok()) return ZDIT_ERR_UNSUPPORTED;
+  return ZDIT_OK;
+}
+
+ZDIT_API zdit_status zdit_stack_forward(const zdit_stack_cfg* cfg, const zdit_stack_weights* w,
+                                        const zdit_stack_inputs* in, float* out, void* workspace,
+                                        size_t workspace_bytes, void* stream) {
+  StackDims d;
+  const zdit_status v = stack_validate(cfg, w, in, out, workspace, &d);
+  if (v != ZDIT_OK) return v;
   Carver c0(nullptr);
   if (workspace_bytes < carve_stack(c0, nullptr, d)) return ZDIT_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   Carver c(workspace);
   StackWs ws;
   carve_stack(c, &ws, d);
-  const int D = d.D, B = d.B, E = d.E;
-  const zdit_block_cfg& bcfg = cfg->block;
+  return stack_run(cfg, w, in, d, ws, out, StackOpts{}, s);
+}
 
-  // token layout: positions and segment offsets of the three sequences
-  launch_stack_layout(d.n_cap, B, in->grid_h, in->grid_w, ws.pos_img, ws.pos_cap, ws.pos_joint, ws.cu_img,
-                      ws.cu_cap, ws.cu_joint, s);
-  launch_rope_table(ws.pos_img, d.T_img, 128, bcfg.rope_axes, bcfg.rope_theta, ws.cos_img, ws.sin_img, s);
-  launch_rope_table(ws.pos_cap, d.T_cap, 128, bcfg.rope_axes, bcfg.rope_theta, ws.cos_cap, ws.sin_cap, s);
-  launch_rope_table(ws.pos_joint, d.T, 128, bcfg.rope_axes, bcfg.rope_theta, ws.cos_joint, ws.sin_joint, s);
+namespace {
+size_t carve_sample(Carver& c, StackWs* ws, float** z, float** vel, const StackDims& d) {
+  carve_stack(c, ws, d);
+  float* zz = c.take<float>((size_t)d.n_img * d.patch_dim);
+  float* vv = c.take<float>((size_t)d.B * d.n_img * d.patch_dim);
+  if (z) *z = zz;
+  if (vel) *vel = vv;
+  return c.off;
+}
 
-  // timestep embedding and every adaLN vector of the forward
-  launch_timestep_embed(in->t, B, E, cfg->t_scale, static_cast<const __nv_bfloat16*>(w->w_t1), w->b_t1,
-                        static_cast<const __nv_bfloat16*>(w->w_t2), w->b_t2, ws.temb, s);
-  for (int i = 0; i < d.nblk; ++i) {
-    const bool ctx = i >= cfg->n_noise_refiner && i < cfg->n_noise_refiner + cfg->n_context_refiner;
-    if (ctx || !(bcfg.flags & ZDIT_F_ADALN)) continue;
-    launch_gemv(static_cast<const __nv_bfloat16*>(w->blocks[i].w_ada), w->blocks[i].b_ada, ws.temb, B, E, 4 * D,
-                ws.mods + (size_t)i * B * 4 * D, s);
-  }
-  launch_gemv(static_cast<const __nv_bfloat16*>(w->w_fada), w->b_fada, ws.temb, B, E, D, ws.fmod, s);
+// stack inputs of the sampler: the latent tokens are shared by every branch
+bool sample_inputs(const zdit_stack_inputs* in, zdit_stack_inputs* in2, float* t_host, const void* some_device_ptr) {
+  if (!in || in->batch <= 0 || in->batch > kMaxBatch) return false;
+  *in2 = *in;
+  for (int b = 0; b < in->batch; ++b) t_host[b] = 0.f;
+  in2->t = t_host;
+  in2->patches = static_cast<const float*>(some_device_ptr);
+  in2->shared_patches = 1;
+  return true;
+}
+}  // namespace
 
-  // image embedder: patches -> bf16 -> Linear(patch_dim, D) + bias
-  for (int b = 0; b < B; ++b)
-    launch_cast_bf16(in->patches + (in->shared_patches ? 0 : (size_t)b * d.n_img * d.patch_dim),
-                     ws.patches16 + (size_t)b * d.n_img * d.patch_dim, (int64_t)d.n_img * d.patch_dim, s);
-  GemmArgs gx{};
-  gx.A = ws.patches16; gx.lda = d.patch_dim; gx.B = w->w_x; gx.ldb = d.patch_dim; gx.M = d.T_img; gx.N = D;
-  gx.K = d.patch_dim; gx.epi = EPI_F32; gx.out = ws.x_img; gx.ldo = D; gx.bias = w->b_x;
-  zdit_status st = launch_gemm(gx, s);
-  if (st != ZDIT_OK) return st;
+ZDIT_API size_t zdit_sample_workspace_bytes(const zdit_stack_cfg* cfg, const zdit_stack_inputs* in) {
+  float t_host[kMaxBatch];
+  zdit_stack_inputs in2;
+  if (!sample_inputs(in, &in2, t_host, reinterpret_cast<const void*>(256))) return 0;
+  StackDims d;
+  if (!stack_dims(cfg, &in2, &d)) return 0;
+  Carver c(nullptr);
+  return carve_sample(c, nullptr, nullptr, nullptr, d);
+}
 
-  // caption embedder: RMSNorm(valid rows) -> Linear(cap_dim, D) + bias; pads <- pad_vec
-  if (cudaMemsetAsync(ws.caps16, 0, (size_t)d.T_cap * d.cap_dim * sizeof(__nv_bfloat16), s) != cudaSuccess)
-    return ZDIT_ERR_CUDA;
-  for (int b = 0; b < B; ++b)
-    if (d.n_valid[b] > 0)
-      launch_norm_modulate_ex(in->cap_feats + (size_t)d.cap_off[b] * d.cap_dim, d.n_valid[b], d.cap_dim,
-                              w->w_capnorm, nullptr, 0, nullptr, 1, 0, 0, bcfg.norm_eps,
-                              ws.caps16 + (size_t)d.cu_cap[b] * d.cap_dim, s);
-  GemmArgs gc{};
-  gc.A = ws.caps16; gc.lda = d.cap_dim; gc.B = w->w_cap; gc.ldb = d.cap_dim; gc.M = d.T_cap; gc.N = D;
-  gc.K = d.cap_dim; gc.epi = EPI_F32; gc.out = ws.x_cap; gc.ldo = D; gc.bias = w->b_cap;
-  st = launch_gemm(gc, s);
-  if (st != ZDIT_OK) return st;
-  for (int b = 0; b < B; ++b)
-    launch_fill_rows(ws.x_cap + (size_t)(d.cu_cap[b] + d.n_valid[b]) * D, D, d.n_cap[b] - d.n_valid[b],
-                     w->pad_vec, s);
-
-  // refiners
-  zdit_varlen v_img{B, ws.cu_img, d.cu_img};
-  zdit_varlen v_cap{B, ws.cu_cap, d.cu_cap};
-  zdit_varlen v_joint{B, ws.cu_joint, d.cu_joint};
-  for (int i = 0; i < d.nblk; ++i) {
-    const bool noise = i < cfg->n_noise_refiner;
-    const bool ctx = !noise && i < cfg->n_noise_refiner + cfg->n_context_refiner;
-    if (!noise && !ctx) continue;
-    zdit_block_cfg bc = bcfg;
-    if (ctx) bc.flags &= ~ZDIT_F_ADALN;
-    const float* mod = ws.mods + (size_t)i * B * 4 * D;
-    st = noise ? run_block(bc, w->blocks[i], v_img, d.T_img, ws.x_img, mod, ws.cos_img, ws.sin_img, ws.blk, s)
-               : run_block(bc, w->blocks[i], v_cap, d.T_cap, ws.x_cap, mod, ws.cos_cap, ws.sin_cap, ws.blk, s);
+ZDIT_API zdit_status zdit_sample(const zdit_stack_cfg* cfg, const zdit_stack_weights* w,
+                                 const zdit_stack_inputs* in, const zdit_sample_cfg* sc, float* latent,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  if (!sc || !latent || !in) return ZDIT_ERR_INVALID_ARG;
+  if (sc->n_steps <= 0 || sc->n_steps > 1000 || in->batch > 2) return ZDIT_ERR_SHAPE;
+  float t_host[kMaxBatch];
+  zdit_stack_inputs in2;
+  if (!sample_inputs(in, &in2, t_host, latent)) return ZDIT_ERR_SHAPE;
+  StackDims d;
+  const zdit_status v = stack_validate(cfg, w, &in2, latent, workspace, &d);
+  if (v != ZDIT_OK) return v;
+  if (d.patch_dim % 4) return ZDIT_ERR_SHAPE;
+  Carver c0(nullptr);
+  if (workspace_bytes < carve_sample(c0, nullptr, nullptr, nullptr, d)) return ZDIT_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Carver c(workspace);
+  StackWs ws;
+  float *z = nullptr, *vel = nullptr;
+  carve_sample(c, &ws, &z, &vel, d);
+  in2.patches = z;
+  const int C = d.patch_dim / 4;
+  const int64_t n = (int64_t)d.n_img * d.patch_dim;
+  launch_patchify(latent, z, C, in->grid_h, in->grid_w, 0, s);
+  StackOpts opts;
+  opts.dedup_noise = sc->dedup_noise != 0 && d.B > 1;
+  for (int i = 0; i < sc->n_steps; ++i) {
+    // sigma_i = 3(1-u)/(3(1-u)+u), u = i / n_steps; the DiT sees t = 1 - sigma_i
+    const double u0 = (double)i / sc->n_steps, u1 = (double)(i + 1) / sc->n_steps;
+    const float s0 = (float)(3.0 * (1.0 - u0) / (3.0 * (1.0 - u0) + u0));
+    const float s1 = (float)(3.0 * (1.0 - u1) / (3.0 * (1.0 - u1) + u1));
+    for (int b = 0; b < d.B; ++b) t_host[b] = 1.0f - s0;
+    opts.context_ready = sc->cache_context != 0 && i > 0;
+    zdit_status st = stack_run(cfg, w, &in2, d, ws, vel, opts, s);
     if (st != ZDIT_OK) return st;
+    launch_euler_cfg(z, vel, d.B > 1 ? vel + n : nullptr, n, sc->guidance, s1 - s0, s);
   }
-  // concatenate each branch as [image | caption]
-  for (int b = 0; b < B; ++b) {
-    if (cudaMemcpyAsync(ws.x_joint + (size_t)d.cu_joint[b] * D, ws.x_img + (size_t)d.cu_img[b] * D,
-                        (size_t)d.n_img * D * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
-      return ZDIT_ERR_CUDA;
-    if (cudaMemcpyAsync(ws.x_joint + (size_t)(d.cu_joint[b] + d.n_img) * D, ws.x_cap + (size_t)d.cu_cap[b] * D,
-                        (size_t)d.n_cap[b] * D * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
-      return ZDIT_ERR_CUDA;
-  }
-  // main blocks; each one's last residual kernel also produces the next block's
-  // pre-attention operand
-  const int first_main = cfg->n_noise_refiner + cfg->n_context_refiner;
-  const bool adaln = bcfg.flags & ZDIT_F_ADALN;
-  for (int i = first_main; i < d.nblk; ++i) {
-    NextNorm nn{};
-    const bool has_next = i + 1 < d.nblk;
-    if (has_next) {
-      nn.w = w->blocks[i + 1].n_attn;
-      nn.scale = adaln ? ws.mods + (size_t)(i + 1) * B * 4 * D : nullptr;
-    }
-    st = run_block(bcfg, w->blocks[i], v_joint, d.T, ws.x_joint, ws.mods + (size_t)i * B * 4 * D, ws.cos_joint,
-                   ws.sin_joint, ws.blk, s, i > first_main, has_next ? &nn : nullptr);
-    if (st != ZDIT_OK) return st;
-  }
-  // final layer on the image rows of each branch
-  for (int b = 0; b < B; ++b) {
-    launch_norm_modulate_ex(ws.x_joint + (size_t)d.cu_joint[b] * D, d.n_img, D, nullptr, ws.fmod + (size_t)b * D, 0,
-                            nullptr, 1, 0, 1, cfg->final_eps, ws.blk.a, s);
-    GemmArgs gf{};
-    gf.A = ws.blk.a; gf.lda = D; gf.B = w->w_final; gf.ldb = D; gf.M = d.n_img; gf.N = d.patch_dim; gf.K = D;
-    gf.epi = EPI_F32; gf.out = out + (size_t)b * d.n_img * d.patch_dim; gf.ldo = d.patch_dim; gf.bias = w->b_final;
-    st = launch_gemm(gf, s);
-    if (st != ZDIT_OK) return st;
-  }
+  launch_patchify(z, latent, C, in->grid_h, in->grid_w, 1, s);
   return cudaGetLastError() == cudaSuccess ? ZDIT_OK : ZDIT_ERR_CUDA;
 }
 

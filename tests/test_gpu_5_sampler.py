@@ -49,3 +49,56 @@ def test_eight_step_sampler_matches_oracle():
     e = errors(host(result), ref)
     print("\nsampler", e)
     assert e["rel_l2"] <= 2e-2, e
+
+
+def _small_setup():
+    d = synth.BlockDims(dim=256, n_heads=2, head_dim=128, ffn_hidden=384)
+    W = synth.stack_weights(9, d, n_noise=2, n_context=2, n_main=2, cap_dim=128)
+    latent = synth.latent_noise(42, (16, 16, 16))
+    caps = synth.randn(9, 300, (46, 128))
+    return d, W, latent, caps
+
+
+@pytest.mark.parametrize("dedup", [False, True])
+def test_sample_entry_point_matches_oracle(dedup):
+    d, W, latent, caps = _small_setup()
+    stack = Z.DeviceStack(W, dims_of(d), 2, 2, 2, patch_dim=64, cap_dim=128)
+    call = Z.StackCall((8, 8), [64, 32], [45, 1], [0.0, 0.0], dev(caps), dev(caps))
+    ws = torch.empty(Z.sample_workspace_bytes(stack, call), dtype=torch.uint8, device="cuda")
+    lat = dev(latent)
+    Z.zdit_sample(stack, call, lat, ws, n_steps=8, guidance=1.0, cache_context=True, dedup_noise=dedup)
+    assert Z.zdit_device_status() == 0
+    cond = {"caps": caps[:45], "n_cap": 64, "n_valid": 45}
+    unc = {"caps": caps[45:], "n_cap": 32, "n_valid": 1}
+    ref = O.sample(latent, cond, unc, W, d, g=1.0, n_steps=8)
+    e = errors(host(lat), ref)
+    print(f"\nzdit_sample dedup={dedup}", e)
+    assert e["rel_l2"] <= 2e-2, e
+
+
+def test_sample_single_branch_guidance_zero():
+    d, W, latent, caps = _small_setup()
+    stack = Z.DeviceStack(W, dims_of(d), 2, 2, 2, patch_dim=64, cap_dim=128)
+    call = Z.StackCall((8, 8), [64], [45], [0.0], dev(caps), dev(caps[:45]))
+    ws = torch.empty(Z.sample_workspace_bytes(stack, call), dtype=torch.uint8, device="cuda")
+    lat = dev(latent)
+    Z.zdit_sample(stack, call, lat, ws, n_steps=8, guidance=0.0)
+    assert Z.zdit_device_status() == 0
+    cond = {"caps": caps[:45], "n_cap": 64, "n_valid": 45}
+    unc = {"caps": caps[45:], "n_cap": 32, "n_valid": 1}
+    ref = O.sample(latent, cond, unc, W, d, g=0.0, n_steps=8)  # g = 0: v = -pos
+    e = errors(host(lat), ref)
+    assert e["rel_l2"] <= 2e-2, e
+
+
+def test_sample_caching_is_bitwise_neutral():
+    # the caption stream has no t dependence: computing it once equals recomputing it
+    d, W, latent, caps = _small_setup()
+    stack = Z.DeviceStack(W, dims_of(d), 2, 2, 2, patch_dim=64, cap_dim=128)
+    call = Z.StackCall((8, 8), [64, 32], [45, 1], [0.0, 0.0], dev(caps), dev(caps))
+    ws = torch.empty(Z.sample_workspace_bytes(stack, call), dtype=torch.uint8, device="cuda")
+    a, b = dev(latent), dev(latent)
+    Z.zdit_sample(stack, call, a, ws, cache_context=True)
+    Z.zdit_sample(stack, call, b, ws, cache_context=False)
+    assert Z.zdit_device_status() == 0
+    assert torch.equal(a, b)
