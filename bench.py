@@ -106,6 +106,8 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ our arm
+SAMPLER_WORKLOAD = ("1024x1024 image: 8-step FlowMatchEuler sampler with negated CFG (g=1) on the "
+                    "cond/uncond pair, 34-block DiT, caption stream computed once (t-independent)")
 BLOCK_WORKLOAD = ("one main DiT block of the 1024x1024 workload: joint cond/uncond sequence 4224 + 4128 "
                   "tokens, width 3840, 30x128 heads, SwiGLU 10240, adaLN + sandwich norm")
 
@@ -180,6 +182,26 @@ def run_ours(args):
             call.set_t([1.0 - s0, 1.0 - s0])
             Z.zdit_stack_forward(stack, call, out, ws)
             Z.zdit_euler_cfg_step(z, out[0], out[1], 1.0, s0, s1)
+    elif args.workload == "sampler":
+        # one 1024x1024 image: 8 sampler steps on the cond/uncond pair in one call
+        stack = build_model(torch, Z, device)
+        latent0 = torch.randn(16, 128, 128, generator=g).to(device)
+        latent = latent0.clone()
+        caps = torch.randn(sum(N_VALIDS), CAP, generator=g).to(device)
+        call = Z.StackCall(GRID, N_CAPS, N_VALIDS, [0.0, 0.0], latent, caps)
+        ws = torch.empty(Z.sample_workspace_bytes(stack, call), dtype=torch.uint8, device=device)
+        inputs, result = [latent], latent
+        n_img_ = GRID[0] * GRID[1]
+        ctx_flops = 2 * (2.0 * sum(N_CAPS) * D * (3 * D + D + 3 * F) + sum(4.0 * D * c * c for c in N_CAPS))
+        noise_flops = 2 * (2.0 * n_img_ * D * (3 * D + D + 3 * F) + 4.0 * D * n_img_ * n_img_)
+        # executed work: 8 forwards, the caption stream once, the noise refiner once per
+        # step for both branches unless deduplicated
+        flops = 8 * forward_flops() - 7 * ctx_flops - (8 * noise_flops if args.dedup else 0)
+
+        def step(i):
+            latent.copy_(latent0)
+            Z.zdit_sample(stack, call, latent, ws, n_steps=8, guidance=1.0, cache_context=True,
+                          dedup_noise=args.dedup)
     else:
         # one main block of the workload: the joint cond/uncond sequence (4224 + 4128)
         from stream_diffusion_transformer_s3_b200 import synth
@@ -292,7 +314,8 @@ def run_ours(args):
             "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": WORKLOAD if args.workload == "stack" else BLOCK_WORKLOAD,
+            "config": {"workload": {"stack": WORKLOAD, "block": BLOCK_WORKLOAD,
+                                    "sampler": SAMPLER_WORKLOAD}[args.workload],
                        "global_batch": 2 * world, "seq_len": [n_img + c for c in N_CAPS],
                        "flops_per_forward": flops, "parallelism": f"replicas x{world}",
                        "l2": ("working set larger than L2 (12.3 GB of bf16 weights streamed per step)" if args.workload == "stack" else "working set larger than L2 (354 MB weights + 128 MB residual + 448 MB activations per block)"),
@@ -307,6 +330,17 @@ def run_ours(args):
         }
         if args.workload == "block":
             res["metric"] = "DiT main-block forward TFLOP/s (1024^2 cond/uncond sequence, bf16, 1 B200)"
+        if args.workload == "sampler":
+            res["metric"] = "s per 1024^2 image, 8-step negated-CFG sampler (bf16, 1 B200)"
+            res["value"] = round(ms / 1e3, 4)
+            res["unit"] = "s/image"
+            res["higher_is_better"] = False
+            res["tflops"] = round(value, 2)
+            res["e2e"] = {"value": round(ms_e2e / 1e3, 4), "unit": "s/image", "ms_per_step": round(ms_e2e, 3),
+                          "h2d_bytes_per_step": res["e2e"]["h2d_bytes_per_step"],
+                          "d2h_bytes_per_step": res["e2e"]["d2h_bytes_per_step"]}
+            res["config"]["workload"] = (SAMPLER_WORKLOAD + (", noise refiner deduplicated across branches"
+                                                             if args.dedup else ""))
         if world == 1 and not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline_block(seconds=None)
         print(json.dumps(res), flush=True)
@@ -383,8 +417,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["stack", "block"], default="stack",
-                    help="stack: the full DiT step (default); block: one main block (for kernel captures)")
+    ap.add_argument("--workload", choices=["stack", "block", "sampler"], default="stack",
+                    help="stack: the full DiT step (default); block: one main block (for kernel captures); "
+                         "sampler: one whole 8-step image per step")
+    ap.add_argument("--dedup", action="store_true",
+                    help="sampler workload: run the noise refiner once for both branches")
     ap.add_argument("--traffic", type=float, default=None,
                     help="dram bytes per launch of the dominant kernel from an ncu capture")
     args = ap.parse_args()

@@ -19,6 +19,8 @@ void launch_norm_modulate_ex(const float* x, int T, int D, const float* w, const
 void launch_gemv(const __nv_bfloat16* W, const float* bias, const float* temb, int B, int E, int rows, float* out,
                  cudaStream_t s);
 void launch_euler_cfg(float* x, const float* vp, const float* vn, int64_t n, float g, float dsig, cudaStream_t s);
+void launch_gemv_batched(const __nv_bfloat16* const* W, const float* const* bias, float* const* out, int nmat,
+                         const float* temb, int B, int E, int rows, cudaStream_t s);
 void launch_rope_table(const int* pos, int64_t T, int head_dim, const int* axes, float theta, float* cs, float* sn,
                        cudaStream_t s);
 void launch_timestep_embed(const float* t_host, int B, int E, float t_scale, const __nv_bfloat16* w1,
@@ -46,6 +48,7 @@ int num_sms() {
 namespace {
 
 constexpr int kMaxBatch = 8;
+constexpr int kMaxBlocks = 256;
 
 bool device_ok() {
   static int ok = -1;
@@ -248,6 +251,7 @@ bool stack_dims(const zdit_stack_cfg* cfg, const zdit_stack_inputs* in, StackDim
   if (in->batch <= 0 || in->batch > kMaxBatch || in->grid_h <= 0 || in->grid_w <= 0) return false;
   if (!in->n_cap || !in->n_valid) return false;
   if (cfg->n_noise_refiner < 0 || cfg->n_context_refiner < 0 || cfg->n_main < 0) return false;
+  if (cfg->n_noise_refiner + cfg->n_context_refiner + cfg->n_main > kMaxBlocks) return false;
   if (cfg->patch_dim <= 0 || cfg->patch_dim % 64 || cfg->cap_dim <= 0 || cfg->cap_dim % 64) return false;
   d->B = in->batch;
   d->n_img = in->grid_h * in->grid_w;
@@ -329,11 +333,21 @@ zdit_status stack_run(const zdit_stack_cfg* cfg, const zdit_stack_weights* w, co
   // timestep embedding and every adaLN vector of the forward
   launch_timestep_embed(in->t, B, E, cfg->t_scale, static_cast<const __nv_bfloat16*>(w->w_t1), w->b_t1,
                         static_cast<const __nv_bfloat16*>(w->w_t2), w->b_t2, ws.temb, s);
-  for (int i = 0; i < d.nblk; ++i) {
-    const bool ctx = i >= cfg->n_noise_refiner && i < cfg->n_noise_refiner + cfg->n_context_refiner;
-    if (ctx || !(bcfg.flags & ZDIT_F_ADALN)) continue;
-    launch_gemv(static_cast<const __nv_bfloat16*>(w->blocks[i].w_ada), w->blocks[i].b_ada, ws.temb, B, E, 4 * D,
-                ws.mods + (size_t)i * B * 4 * D, s);
+  {
+    // every adaLN projection of the forward in one launch
+    const __nv_bfloat16* Ws[kMaxBlocks];
+    const float* bs[kMaxBlocks];
+    float* outs[kMaxBlocks];
+    int nm = 0;
+    for (int i = 0; i < d.nblk && (bcfg.flags & ZDIT_F_ADALN); ++i) {
+      const bool ctx = i >= cfg->n_noise_refiner && i < cfg->n_noise_refiner + cfg->n_context_refiner;
+      if (ctx) continue;
+      Ws[nm] = static_cast<const __nv_bfloat16*>(w->blocks[i].w_ada);
+      bs[nm] = w->blocks[i].b_ada;
+      outs[nm] = ws.mods + (size_t)i * B * 4 * D;
+      ++nm;
+    }
+    if (nm > 0) launch_gemv_batched(Ws, bs, outs, nm, ws.temb, B, E, 4 * D, s);
   }
   launch_gemv(static_cast<const __nv_bfloat16*>(w->w_fada), w->b_fada, ws.temb, B, E, D, ws.fmod, s);
 

@@ -50,6 +50,7 @@ zdit_status read_and_clear_device_error() {
 namespace {
 
 constexpr int RT = 256;  // threads per row CTA
+constexpr int kGemvBatchMax = 40;
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -257,6 +258,62 @@ __global__ void __launch_bounds__(256) adaln_gemv_kernel(const __nv_bfloat16* __
     if (b < B) {
       const float s = warp_sum(acc[b]);
       if (lane == 0) out[(size_t)b * rows + r] = s + (bias != nullptr ? bias[r] : 0.f);
+    }
+  }
+}
+
+// Several GEMVs of the same shape in one launch (every adaLN projection of a forward):
+// blockIdx.y selects the matrix.
+struct GemvBatch {
+  const __nv_bfloat16* W[kGemvBatchMax];
+  const float* bias[kGemvBatchMax];
+  float* out[kGemvBatchMax];
+};
+
+__global__ void __launch_bounds__(256) adaln_gemv_batched_kernel(const __grid_constant__ GemvBatch gb,
+                                                                 const float* __restrict__ temb, int B, int E,
+                                                                 int rows) {
+  extern __shared__ float st[];  // [B, E]
+  for (int i = threadIdx.x; i < B * E; i += blockDim.x) st[i] = temb[i];
+  __syncthreads();
+  const int m = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const __nv_bfloat16* W = gb.W[m];
+  const float* bias = gb.bias[m];
+  float* out = gb.out[m];
+  // each warp: 4 rows, all loads issued before the reductions
+  const int r0 = (blockIdx.x * 8 + warp) * 4;
+  float acc[4][8];
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+#pragma unroll
+    for (int b = 0; b < 8; ++b) acc[q][b] = 0.f;
+  for (int e0 = lane * 8; e0 < E; e0 += 256) {
+    uint4 u[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      u[q] = r0 + q < rows ? *reinterpret_cast<const uint4*>(W + (size_t)(r0 + q) * E + e0) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&u[q]);
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        if (b < B) {
+          const float* tb = st + b * E + e0;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc[q][b] += __bfloat162float(h[j]) * tb[j];
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+      if (b < B) {
+        const float v = warp_sum(acc[q][b]);
+        if (lane == 0 && r0 + q < rows) out[(size_t)b * rows + r0 + q] = v + (bias != nullptr ? bias[r0 + q] : 0.f);
+      }
     }
   }
 }
@@ -471,6 +528,22 @@ void launch_gemv(const __nv_bfloat16* W, const float* bias, const float* temb, i
                  cudaStream_t s) {
   ProfScope ps(PROF_GEMV, 2.0 * rows * (double)E * B, 2.0 * rows * (double)E + 4.0 * rows * (B + 1.0), s);
   adaln_gemv_kernel<<<(rows + 7) / 8, 256, (size_t)B * E * sizeof(float), s>>>(W, bias, temb, B, E, rows, out);
+}
+
+void launch_gemv_batched(const __nv_bfloat16* const* W, const float* const* bias, float* const* out, int nmat,
+                         const float* temb, int B, int E, int rows, cudaStream_t s) {
+  for (int m0 = 0; m0 < nmat; m0 += kGemvBatchMax) {
+    const int nm = nmat - m0 < kGemvBatchMax ? nmat - m0 : kGemvBatchMax;
+    GemvBatch gb{};
+    for (int i = 0; i < nm; ++i) {
+      gb.W[i] = W[m0 + i];
+      gb.bias[i] = bias[m0 + i];
+      gb.out[i] = out[m0 + i];
+    }
+    ProfScope ps(PROF_GEMV, 2.0 * rows * (double)E * B * nm, (2.0 * rows * (double)E + 4.0 * rows * (B + 1.0)) * nm, s);
+    dim3 grid((rows + 31) / 32, nm);
+    adaln_gemv_batched_kernel<<<grid, 256, (size_t)B * E * sizeof(float), s>>>(gb, temb, B, E, rows);
+  }
 }
 
 void launch_euler_cfg(float* x, const float* vp, const float* vn, int64_t n, float g, float dsig, cudaStream_t s) {
