@@ -179,6 +179,14 @@ __global__ void __launch_bounds__(RT) residual_kernel(ResidParams p) {
     }
     ss += y[i].x * y[i].x + y[i].y * y[i].y + y[i].z * y[i].z + y[i].w * y[i].w;
   }
+  // the residual row does not depend on the reduction: load it now so both streams
+  // are in flight together
+  float4 xv[MAXV];
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int idx = (i * RT + threadIdx.x) * 4;
+    xv[i] = idx < p.D ? *reinterpret_cast<const float4*>(xr + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   float r = 1.f;
   if (p.post_w != nullptr) r = 1.0f / sqrtf(block_sum(ss, sh) / p.D + p.eps);
   const int br = branch_of(p.cu, p.batch, t);
@@ -188,7 +196,7 @@ __global__ void __launch_bounds__(RT) residual_kernel(ResidParams p) {
   for (int i = 0; i < MAXV; ++i) {
     const int idx = (i * RT + threadIdx.x) * 4;
     if (idx < p.D) {
-      float4 x4 = *reinterpret_cast<const float4*>(xr + idx);
+      float4 x4 = xv[i];
       float4 w4 = p.post_w != nullptr ? *reinterpret_cast<const float4*>(p.post_w + idx)
                                       : make_float4(1.f, 1.f, 1.f, 1.f);
       float4 g4 = g != nullptr ? *reinterpret_cast<const float4*>(g + idx) : make_float4(1.f, 1.f, 1.f, 1.f);
@@ -281,8 +289,8 @@ __global__ void __launch_bounds__(256) adaln_gemv_batched_kernel(const __grid_co
   const __nv_bfloat16* W = gb.W[m];
   const float* bias = gb.bias[m];
   float* out = gb.out[m];
-  // each warp: 4 rows, all loads issued before the reductions
-  const int r0 = (blockIdx.x * 8 + warp) * 4;
+  // each warp: 4 rows at a time, all loads of a group issued before the reductions
+  for (int r0 = (blockIdx.x * 8 + warp) * 16; r0 < (blockIdx.x * 8 + warp) * 16 + 16; r0 += 4) {
   float acc[4][8];
 #pragma unroll
   for (int q = 0; q < 4; ++q)
@@ -315,6 +323,7 @@ __global__ void __launch_bounds__(256) adaln_gemv_batched_kernel(const __grid_co
         if (lane == 0 && r0 + q < rows) out[(size_t)b * rows + r0 + q] = v + (bias != nullptr ? bias[r0 + q] : 0.f);
       }
     }
+  }
   }
 }
 
@@ -541,7 +550,7 @@ void launch_gemv_batched(const __nv_bfloat16* const* W, const float* const* bias
       gb.out[i] = out[m0 + i];
     }
     ProfScope ps(PROF_GEMV, 2.0 * rows * (double)E * B * nm, (2.0 * rows * (double)E + 4.0 * rows * (B + 1.0)) * nm, s);
-    dim3 grid((rows + 31) / 32, nm);
+    dim3 grid((rows + 127) / 128, nm);
     adaln_gemv_batched_kernel<<<grid, 256, (size_t)B * E * sizeof(float), s>>>(gb, temb, B, E, rows);
   }
 }
