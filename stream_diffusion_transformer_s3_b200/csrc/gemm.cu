@@ -50,17 +50,24 @@ struct KParams {
   const float* kn;
   float eps;
   int dim;
-  int num_m, num_n, num_k, group_m, raster;
+  int num_m, num_n, num_k, group_m, group_n, raster;
   int* err;
 };
 
-// Tile order of the persistent loop.  raster 0: M fastest inside bands of group_m
-// M-tiles; raster 1: N fastest.  The host picks the order that keeps the smaller
-// operand resident in L2 while the larger one streams from HBM once.
+// Tile order of the persistent loop.  raster 0: bands of group_m M-tiles, M fastest
+// inside a band (the band of A stays in L2 while B streams); raster 1: bands of
+// group_n N-tiles, N fastest inside a band (the band of B stays in L2 while A
+// streams).  The host sizes the band to a fraction of L2 and picks the order with
+// less estimated HBM traffic.
 __device__ __forceinline__ void tile_coords(int t, const KParams& p, int& mb, int& nb) {
   if (p.raster == 1) {
-    mb = t / p.num_n;
-    nb = t - mb * p.num_n;
+    const int group = p.group_n * p.num_m;
+    const int g = t / group;
+    const int first = g * p.group_n;
+    const int gn = min(p.num_n - first, p.group_n);
+    const int r = t - g * group;
+    nb = first + r % gn;
+    mb = r / gn;
     return;
   }
   const int group = p.group_m * p.num_n;
@@ -609,12 +616,22 @@ zdit_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
   kp.num_m = pair ? (a.M + 255) / 256 : (a.M + BM - 1) / BM;
   kp.num_n = (a.N + BN - 1) / BN;
   kp.num_k = (a.K + BK - 1) / BK;
-  // Whichever operand is smaller stays L2-resident: with A (activations) smaller,
-  // sweep every M tile of an N column before moving on (B read from HBM once, A
-  // re-read from L2); otherwise sweep N fastest (A read once, B re-read from L2).
-  const double a_bytes = 2.0 * a.M * a.K, b_bytes = 2.0 * a.N * a.K;
-  kp.raster = a_bytes <= b_bytes ? 0 : 1;
-  kp.group_m = kp.num_m;
+  // L2-aware raster: a band of tiles of one operand (about 32 MB, well inside one
+  // die's share of the L2) stays resident while the other operand streams; the
+  // streamed operand is re-read once per band.
+  {
+    const double band = 32.0 * (1 << 20);
+    const double a_tile = 2.0 * (pair ? 256 : BM) * a.K, b_tile = 2.0 * BN * a.K;
+    const double a_all = 2.0 * a.M * a.K, b_all = 2.0 * a.N * a.K;
+    int gm = (int)(band / a_tile), gn = (int)(band / b_tile);
+    gm = gm < 1 ? 1 : (gm > kp.num_m ? kp.num_m : gm);
+    gn = gn < 1 ? 1 : (gn > kp.num_n ? kp.num_n : gn);
+    const double traffic_m = a_all + b_all * ((kp.num_m + gm - 1) / gm);
+    const double traffic_n = b_all + a_all * ((kp.num_n + gn - 1) / gn);
+    kp.group_m = gm;
+    kp.group_n = gn;
+    kp.raster = traffic_m <= traffic_n ? 0 : 1;
+  }
   kp.err = device_error_ptr();
   const int tiles = kp.num_m * kp.num_n;
   int grid = tiles < num_sms() ? tiles : num_sms();
