@@ -28,6 +28,10 @@
 #include "internal.h"
 #include "ptx.cuh"
 
+#ifndef ZDIT_L2_BAND_MB
+#define ZDIT_L2_BAND_MB 32
+#endif
+
 namespace zdit {
 
 namespace {
@@ -620,7 +624,7 @@ zdit_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
   // die's share of the L2) stays resident while the other operand streams; the
   // streamed operand is re-read once per band.
   {
-    const double band = 32.0 * (1 << 20);
+    const double band = (double)ZDIT_L2_BAND_MB * (1 << 20);
     const double a_tile = 2.0 * (pair ? 256 : BM) * a.K, b_tile = 2.0 * BN * a.K;
     const double a_all = 2.0 * a.M * a.K, b_all = 2.0 * a.N * a.K;
     int gm = (int)(band / a_tile), gn = (int)(band / b_tile);
