@@ -53,6 +53,21 @@ def forward_flops() -> float:
     return f
 
 
+# DRAM bytes per launch of the dominant kernel (gate/up GEMM of a main block, 8352 x 20480
+# x 3840), from one ncu capture (profiles/gemm_gate_up_swiglu_block_1024.md), valid for the
+# GEMM sources with this hash only; any change to them makes the figure stale (reported null).
+NCU_TRAFFIC = {"kernel": "gemm_gate_up_swiglu", "bytes": 448198144 + 156702720, "src_hash": "5d5279801f9e4f66"}
+
+
+def gemm_src_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("gemm.cu", "ptx.cuh", "internal.h"):
+        with open(os.path.join(ROOT, "stream_diffusion_transformer_s3_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -294,7 +309,10 @@ def run_ours(args):
             achieved = k["flops"] / (k["total_ms"] * 1e-3) / 1e12
             roofline = {"kernel": name, "bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
                         "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                        "peak_source": f"{peak_src} bf16 {peak_kind}", "traffic": args.traffic,
+                        "peak_source": f"{peak_src} bf16 {peak_kind}",
+                        "traffic": (args.traffic if args.traffic is not None else
+                                    NCU_TRAFFIC["bytes"] if (name == NCU_TRAFFIC["kernel"] and
+                                                             gemm_src_hash() == NCU_TRAFFIC["src_hash"]) else None),
                         "launches_per_step": k["launches"] / args.steps,
                         "ms_per_launch": k["total_ms"] / k["launches"]}
     kern_summary = {}
