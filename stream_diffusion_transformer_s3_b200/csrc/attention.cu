@@ -215,31 +215,40 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else if (warp == WARP_MMA && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
+    // Each UMMA here is only 64 tensor clocks of work, so the issuing thread must do
+    // almost nothing per instruction: every shared-memory descriptor is precomputed
+    // (a descriptor is linear in the address: desc(addr + off) = desc(addr) + off / 16).
     const uint32_t id_s = idesc_bf16_f32(TILE, TILE);             // Q, K both K-major
     const uint32_t id_o = idesc_bf16_f32(TILE, HD, false, true);  // P from TMEM, V MN-major
-    const uint32_t aQ = smem_u32(smem + OFF_Q);
+    uint64_t dq[2], dk[2], dv[2];
+    for (int t = 0; t < 2; ++t) dq[t] = sdesc_kmajor_sw128(smem_u32(smem + OFF_Q + t * TILE_BYTES));
+    for (int i = 0; i < 2; ++i) dk[i] = sdesc_kmajor_sw128(smem_u32(smem + OFF_K + i * TILE_BYTES));
+    for (int i = 0; i < 2; ++i) dv[i] = sdesc_mnmajor_sw128(smem_u32(smem + OFF_V + i * TILE_BYTES), HALF, 1024);
+    // K step k of a K-major 128-byte-swizzled tile: (k / 4) 64-column halves + (k % 4) 32-byte slices
+    auto koff = [](int k) -> uint64_t { return (uint64_t)(((k >> 2) * HALF + (k & 3) * 32) >> 4); };
+    // K step k of the MN-major V tile: 16 key rows of 128 bytes
+    auto voff = [](int k) -> uint64_t { return (uint64_t)((k * 16 * 128) >> 4); };
+    const uint32_t tm_s[2] = {tmem, tmem + 128};
+    const uint32_t tm_o[2] = {tmem + 256, tmem + 384};
     // O_t += P_t V_i ; P_t read from TMEM columns [t*128, t*128 + 64)
     auto issue_pv = [&](int t, int i) -> bool {
       if (!mbar_wait(&p_full[t], i & 1, abort_flag, p.err)) return false;
       if (t == 0 && !mbar_wait(&v_full[i & 1], (i >> 1) & 1, abort_flag, p.err)) return false;
       tc_fence_after();
-      const uint32_t aV = smem_u32(smem + OFF_V + (i & 1) * TILE_BYTES);
+      const uint64_t vb = dv[i & 1];
+      const uint32_t d = tm_o[t], pa = tm_s[t];
+      umma_bf16_ts(d, pa, vb, id_o, i != 0 ? 1u : 0u);
 #pragma unroll
-      for (int k = 0; k < TILE / 16; ++k)
-        umma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + k * 8,
-                     sdesc_mnmajor_sw128(aV + k * 16 * 128, HALF, 1024), id_o, (i | k) != 0 ? 1u : 0u);
+      for (int k = 1; k < TILE / 16; ++k) umma_bf16_ts(d, pa + k * 8, vb + voff(k), id_o, 1u);
       return true;
     };
     // S_t = Q_t K_j^T into TMEM columns [t*128, t*128 + 128)
     auto issue_s = [&](int t, int j) {
-      const uint32_t aK = smem_u32(smem + OFF_K + (j & 1) * TILE_BYTES);
-      const uint32_t aQt = aQ + t * TILE_BYTES;
+      const uint64_t kb = dk[j & 1], qb = dq[t];
+      const uint32_t d = tm_s[t];
+      umma_bf16_ss(d, qb, kb, id_s, 0u);
 #pragma unroll
-      for (int k = 0; k < HD / 16; ++k) {
-        const uint32_t off = (k >> 2) * HALF + (k & 3) * 32;
-        umma_bf16_ss(tmem + t * 128, sdesc_kmajor_sw128(aQt + off), sdesc_kmajor_sw128(aK + off), id_s,
-                     k != 0 ? 1u : 0u);
-      }
+      for (int k = 1; k < HD / 16; ++k) umma_bf16_ss(d, qb + koff(k), kb + koff(k), id_s, 1u);
       umma_commit(&s_full[t]);
     };
     bool ok = mbar_wait(q_full, 0, abort_flag, p.err);
