@@ -68,6 +68,19 @@ def gemm_src_hash() -> str:
     return h.hexdigest()[:16]
 
 
+def aggregate_ranks(ms, ms_e2e, flops, world, dist=None, device="cpu"):
+    """Whole-job rates of `world` independent replicas: each rank ran the same work;
+    the job time is the slowest rank's (max over ranks, through the process group)."""
+    import torch
+    if world > 1 and dist is not None:
+        t = torch.tensor([ms, ms_e2e], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, ms_e2e = float(t[0]), float(t[1])
+    value = world * flops / (ms * 1e-3) / 1e12
+    value_e2e = world * flops / (ms_e2e * 1e-3) / 1e12
+    return ms, ms_e2e, value, value_e2e
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -288,12 +301,7 @@ def run_ours(args):
     barrier()
     ms_e2e = e0.elapsed_time(e1) / args.steps
 
-    if world > 1:
-        t = torch.tensor([ms, ms_e2e], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, ms_e2e = float(t[0]), float(t[1])
-    value = world * flops / (ms * 1e-3) / 1e12
-    value_e2e = world * flops / (ms_e2e * 1e-3) / 1e12
+    ms, ms_e2e, value, value_e2e = aggregate_ranks(ms, ms_e2e, flops, world, dist if world > 1 else None, device)
 
     peaks, peak_src = load_peaks()
     # a timed region of a few seconds or more runs under the power cap: compare with
