@@ -5,7 +5,7 @@
 //                   final layer; plain RMSNorm for the caption embedder)
 //   residual      : x += gate_b * PostNorm(y) (y bf16), optionally fused with the
 //                   next pre-norm so x is read once per step
-//   adaln_gemv    : m_b = W_ada temb_b + b_ada (weight-streaming GEMV)
+//   adaln_gemv    : m_b = W_ada temb_b + b_ada (weight-streaming GEMV, 8 rows per warp)
 //   euler_cfg     : x += (sigma_next - sigma_cur) * -(pos + g (pos - neg))
 //   rope_table    : per-token cos/sin of the 3-axis rotary angles
 //   timestep_embed, patchify / unpatchify, casts and row fills
@@ -230,46 +230,6 @@ __global__ void __launch_bounds__(RT) residual_kernel(ResidParams p) {
   }
 }
 
-// out[b * rows + r] = sum_e W[r, e] * temb[b, e] + bias[r]; one warp per row r,
-// 16-byte weight loads, temb staged in shared memory.
-__global__ void __launch_bounds__(256) adaln_gemv_kernel(const __nv_bfloat16* __restrict__ W,
-                                                         const float* __restrict__ bias,
-                                                         const float* __restrict__ temb, int B, int E, int rows,
-                                                         float* __restrict__ out) {
-  extern __shared__ float st[];  // [B, E]
-  for (int i = threadIdx.x; i < B * E; i += blockDim.x) st[i] = temb[i];
-  __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = blockIdx.x * 8 + warp;
-  if (r >= rows) return;
-  float acc[8];
-#pragma unroll
-  for (int b = 0; b < 8; ++b) acc[b] = 0.f;
-  const __nv_bfloat16* wr = W + (size_t)r * E;
-  for (int e0 = lane * 8; e0 < E; e0 += 256) {
-    const uint4 u = *reinterpret_cast<const uint4*>(wr + e0);
-    const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&u);
-    float w[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) w[j] = __bfloat162float(h[j]);
-#pragma unroll
-    for (int b = 0; b < 8; ++b) {
-      if (b < B) {
-        const float* tb = st + b * E + e0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[b] += w[j] * tb[j];
-      }
-    }
-  }
-#pragma unroll
-  for (int b = 0; b < 8; ++b) {
-    if (b < B) {
-      const float s = warp_sum(acc[b]);
-      if (lane == 0) out[(size_t)b * rows + r] = s + (bias != nullptr ? bias[r] : 0.f);
-    }
-  }
-}
-
 // Several GEMVs of the same shape in one launch (every adaLN projection of a forward):
 // blockIdx.y selects the matrix.
 struct GemvBatch {
@@ -278,52 +238,76 @@ struct GemvBatch {
   float* out[kGemvBatchMax];
 };
 
-__global__ void __launch_bounds__(256) adaln_gemv_batched_kernel(const __grid_constant__ GemvBatch gb,
-                                                                 const float* __restrict__ temb, int B, int E,
-                                                                 int rows) {
-  extern __shared__ float st[];  // [B, E]
-  for (int i = threadIdx.x; i < B * E; i += blockDim.x) st[i] = temb[i];
-  __syncthreads();
+// Weight-streaming GEMV of the adaLN projections: out_m[b, r] = sum_e W_m[r, e] temb[b, e]
+// + bias_m[r].  A warp owns 8 rows and keeps their 16-byte weight loads in flight together
+// (the weights are read once, so the loads bypass L1); lane l covers columns [8l, 8l + 8)
+// of every 256-column chunk and holds the matching temb slice in registers.
+template <int B>
+__global__ void __launch_bounds__(128) adaln_gemv_kernel(const __grid_constant__ GemvBatch gb,
+                                                         const float* __restrict__ temb, int E, int rows) {
   const int m = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r0 = (blockIdx.x * 4 + warp) * 8;
+  if (r0 >= rows) return;
   const __nv_bfloat16* W = gb.W[m];
+  float acc[8][B];
+#pragma unroll
+  for (int r = 0; r < 8; ++r)
+#pragma unroll
+    for (int b = 0; b < B; ++b) acc[r][b] = 0.f;
+  for (int e0 = lane * 8; e0 < E; e0 += 256) {
+    uint4 u[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+      u[r] = r0 + r < rows ? __ldcs(reinterpret_cast<const uint4*>(W + (size_t)(r0 + r) * E + e0))
+                           : make_uint4(0u, 0u, 0u, 0u);
+    float t[B][8];
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      const float4 lo = __ldg(reinterpret_cast<const float4*>(temb + (size_t)b * E + e0));
+      const float4 hi = __ldg(reinterpret_cast<const float4*>(temb + (size_t)b * E + e0 + 4));
+      t[b][0] = lo.x; t[b][1] = lo.y; t[b][2] = lo.z; t[b][3] = lo.w;
+      t[b][4] = hi.x; t[b][5] = hi.y; t[b][6] = hi.z; t[b][7] = hi.w;
+    }
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&u[r]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float w = __bfloat162float(h[j]);
+#pragma unroll
+        for (int b = 0; b < B; ++b) acc[r][b] = fmaf(w, t[b][j], acc[r][b]);
+      }
+    }
+  }
   const float* bias = gb.bias[m];
   float* out = gb.out[m];
-  // each warp: 4 rows at a time, all loads of a group issued before the reductions
-  for (int r0 = (blockIdx.x * 8 + warp) * 16; r0 < (blockIdx.x * 8 + warp) * 16 + 16; r0 += 4) {
-  float acc[4][8];
 #pragma unroll
-  for (int q = 0; q < 4; ++q)
+  for (int r = 0; r < 8; ++r) {
 #pragma unroll
-    for (int b = 0; b < 8; ++b) acc[q][b] = 0.f;
-  for (int e0 = lane * 8; e0 < E; e0 += 256) {
-    uint4 u[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      u[q] = r0 + q < rows ? *reinterpret_cast<const uint4*>(W + (size_t)(r0 + q) * E + e0) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&u[q]);
-#pragma unroll
-      for (int b = 0; b < 8; ++b) {
-        if (b < B) {
-          const float* tb = st + b * E + e0;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) acc[q][b] += __bfloat162float(h[j]) * tb[j];
-        }
-      }
+    for (int b = 0; b < B; ++b) {
+      const float v = warp_sum(acc[r][b]);
+      if (lane == 0 && r0 + r < rows) out[(size_t)b * rows + r0 + r] = v + (bias != nullptr ? bias[r0 + r] : 0.f);
     }
   }
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-#pragma unroll
-    for (int b = 0; b < 8; ++b) {
-      if (b < B) {
-        const float v = warp_sum(acc[q][b]);
-        if (lane == 0 && r0 + q < rows) out[(size_t)b * rows + r0 + q] = v + (bias != nullptr ? bias[r0 + q] : 0.f);
-      }
-    }
-  }
+}
+
+template <int B>
+void launch_gemv_b(const GemvBatch& gb, int nm, const float* temb, int E, int rows, cudaStream_t s) {
+  dim3 grid((rows + 31) / 32, nm);
+  adaln_gemv_kernel<B><<<grid, 128, 0, s>>>(gb, temb, E, rows);
+}
+
+void launch_gemv_any(const GemvBatch& gb, int nm, const float* temb, int B, int E, int rows, cudaStream_t s) {
+  switch (B) {
+    case 1: launch_gemv_b<1>(gb, nm, temb, E, rows, s); break;
+    case 2: launch_gemv_b<2>(gb, nm, temb, E, rows, s); break;
+    case 3: launch_gemv_b<3>(gb, nm, temb, E, rows, s); break;
+    case 4: launch_gemv_b<4>(gb, nm, temb, E, rows, s); break;
+    case 5: launch_gemv_b<5>(gb, nm, temb, E, rows, s); break;
+    case 6: launch_gemv_b<6>(gb, nm, temb, E, rows, s); break;
+    case 7: launch_gemv_b<7>(gb, nm, temb, E, rows, s); break;
+    default: launch_gemv_b<8>(gb, nm, temb, E, rows, s); break;
   }
 }
 
@@ -536,7 +520,11 @@ void launch_residual(const ResidArgs& a, cudaStream_t s) {
 void launch_gemv(const __nv_bfloat16* W, const float* bias, const float* temb, int B, int E, int rows, float* out,
                  cudaStream_t s) {
   ProfScope ps(PROF_GEMV, 2.0 * rows * (double)E * B, 2.0 * rows * (double)E + 4.0 * rows * (B + 1.0), s);
-  adaln_gemv_kernel<<<(rows + 7) / 8, 256, (size_t)B * E * sizeof(float), s>>>(W, bias, temb, B, E, rows, out);
+  GemvBatch gb{};
+  gb.W[0] = W;
+  gb.bias[0] = bias;
+  gb.out[0] = out;
+  launch_gemv_any(gb, 1, temb, B, E, rows, s);
 }
 
 void launch_gemv_batched(const __nv_bfloat16* const* W, const float* const* bias, float* const* out, int nmat,
@@ -550,8 +538,7 @@ void launch_gemv_batched(const __nv_bfloat16* const* W, const float* const* bias
       gb.out[i] = out[m0 + i];
     }
     ProfScope ps(PROF_GEMV, 2.0 * rows * (double)E * B * nm, (2.0 * rows * (double)E + 4.0 * rows * (B + 1.0)) * nm, s);
-    dim3 grid((rows + 127) / 128, nm);
-    adaln_gemv_batched_kernel<<<grid, 256, (size_t)B * E * sizeof(float), s>>>(gb, temb, B, E, rows);
+    launch_gemv_any(gb, nm, temb, B, E, rows, s);
   }
 }
 
