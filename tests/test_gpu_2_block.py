@@ -59,3 +59,13 @@ def test_config2_full_width_block():
 def test_config2_full_width_block_qk_norm_no_sandwich():
     case = synth.block_case(1, synth.FULL, 16, 16, [64, 32], [45, 1], x_max=6.7e3, qk_norm=True)
     _check(case, synth.FULL, O.Flags(sandwich=False, qk_norm=True))
+
+
+@pytest.mark.parametrize("n_caps,n_valids", [
+    ([32, 48, 16], [25, 30, 1]),           # three branches
+    ([16] * 8, [16, 9, 1, 16, 3, 12, 7, 1]),  # the largest batch the library takes
+])
+def test_tiny_block_more_branches(n_caps, n_valids):
+    # every branch has its own adaLN vector: covers the batched projection for B = 3 and 8
+    case = synth.block_case(7, synth.TINY, 8, 8, n_caps, n_valids)
+    _check(case, synth.TINY, O.Flags())
