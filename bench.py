@@ -229,7 +229,7 @@ def run_ours(args):
         def step(i):
             latent.copy_(latent0)
             Z.zdit_sample(stack, call, latent, ws, n_steps=8, guidance=1.0, cache_context=True,
-                          dedup_noise=args.dedup)
+                          dedup_noise=args.dedup, use_graph=args.graph)
     else:
         # one main block of the workload: the joint cond/uncond sequence (4224 + 4128)
         from stream_diffusion_transformer_s3_b200 import synth
@@ -368,7 +368,8 @@ def run_ours(args):
                           "h2d_bytes_per_step": res["e2e"]["h2d_bytes_per_step"],
                           "d2h_bytes_per_step": res["e2e"]["d2h_bytes_per_step"]}
             res["config"]["workload"] = (SAMPLER_WORKLOAD + (", noise refiner deduplicated across branches"
-                                                             if args.dedup else ""))
+                                                             if args.dedup else "")
+                                         + (", captured as one CUDA graph and replayed" if args.graph else ""))
         if world == 1 and not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline_block(seconds=None)
         print(json.dumps(res), flush=True)
@@ -448,6 +449,8 @@ def main():
     ap.add_argument("--workload", choices=["stack", "block", "sampler"], default="stack",
                     help="stack: the full DiT step (default); block: one main block (for kernel captures); "
                          "sampler: one whole 8-step image per step")
+    ap.add_argument("--graph", action="store_true",
+                    help="sampler workload: the whole image as one captured CUDA graph, replayed")
     ap.add_argument("--dedup", action="store_true",
                     help="sampler workload: run the noise refiner once for both branches")
     ap.add_argument("--traffic", type=float, default=None,

@@ -68,7 +68,7 @@ class StackInputs(C.Structure):
 
 class SampleCfg(C.Structure):
     _fields_ = [("n_steps", C.c_int32), ("guidance", C.c_float), ("cache_context", C.c_int32),
-                ("dedup_noise", C.c_int32)]
+                ("dedup_noise", C.c_int32), ("use_graph", C.c_int32)]
 
 
 class ProfileEntry(C.Structure):
@@ -368,9 +368,11 @@ def sample_workspace_bytes(stack: DeviceStack, call: StackCall) -> int:
 
 
 def zdit_sample(stack: DeviceStack, call: StackCall, latent, workspace, n_steps=8, guidance=1.0,
-                cache_context=True, dedup_noise=False, stream=None):
-    """In-place 8-step negated-CFG FlowMatchEuler sampling of `latent` [C, 2h, 2w]."""
-    sc = SampleCfg(n_steps, guidance, 1 if cache_context else 0, 1 if dedup_noise else 0)
+                cache_context=True, dedup_noise=False, use_graph=False, stream=None):
+    """In-place 8-step negated-CFG FlowMatchEuler sampling of `latent` [C, 2h, 2w].
+    use_graph: capture the launch sequence as one CUDA graph and replay it on later calls
+    with the same arguments."""
+    sc = SampleCfg(n_steps, guidance, 1 if cache_context else 0, 1 if dedup_noise else 0, 1 if use_graph else 0)
     _check(lib().zdit_sample(C.byref(stack.cfg), C.byref(stack.wstruct), C.byref(call.struct), C.byref(sc),
                              _ptr(latent), _ptr(workspace), workspace.numel() * workspace.element_size(),
                              _stream(stream)), "zdit_sample")

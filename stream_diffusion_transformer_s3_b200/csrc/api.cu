@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "internal.h"
 
@@ -441,7 +442,7 @@ using namespace zdit;
 
 extern "C" {
 
-ZDIT_API int32_t zdit_version(void) { return 100; }
+ZDIT_API int32_t zdit_version(void) { return 200; }
 
 ZDIT_API const char* zdit_status_string(zdit_status s) {
   switch (s) {
@@ -556,6 +557,61 @@ bool sample_inputs(const zdit_stack_inputs* in, zdit_stack_inputs* in2, float* t
 }
 }  // namespace
 
+}  // extern "C"
+
+namespace zdit {
+namespace {
+
+// The sampler's launch sequence: patchify, n_steps x (stack forward + CFG-Euler update),
+// unpatchify.  Inputs are validated by the caller.
+zdit_status sample_run(const zdit_stack_cfg* cfg, const zdit_stack_weights* w, const zdit_stack_inputs* in,
+                       const zdit_sample_cfg* sc, float* latent, void* workspace, const StackDims& d,
+                       zdit_stack_inputs& in2, float* t_host, cudaStream_t s) {
+  Carver c(workspace);
+  StackWs ws;
+  float *z = nullptr, *vel = nullptr;
+  carve_sample(c, &ws, &z, &vel, d);
+  in2.patches = z;
+  const int C = d.patch_dim / 4;
+  const int64_t n = (int64_t)d.n_img * d.patch_dim;
+  launch_patchify(latent, z, C, in->grid_h, in->grid_w, 0, s);
+  StackOpts opts;
+  opts.dedup_noise = sc->dedup_noise != 0 && d.B > 1;
+  for (int i = 0; i < sc->n_steps; ++i) {
+    // sigma_i = 3(1-u)/(3(1-u)+u), u = i / n_steps; the DiT sees t = 1 - sigma_i
+    const double u0 = (double)i / sc->n_steps, u1 = (double)(i + 1) / sc->n_steps;
+    const float s0 = (float)(3.0 * (1.0 - u0) / (3.0 * (1.0 - u0) + u0));
+    const float s1 = (float)(3.0 * (1.0 - u1) / (3.0 * (1.0 - u1) + u1));
+    for (int b = 0; b < d.B; ++b) t_host[b] = 1.0f - s0;
+    opts.context_ready = sc->cache_context != 0 && i > 0;
+    zdit_status st = stack_run(cfg, w, &in2, d, ws, vel, opts, s);
+    if (st != ZDIT_OK) return st;
+    launch_euler_cfg(z, vel, d.B > 1 ? vel + n : nullptr, n, sc->guidance, s1 - s0, s);
+  }
+  launch_patchify(z, latent, C, in->grid_h, in->grid_w, 1, s);
+  return cudaGetLastError() == cudaSuccess ? ZDIT_OK : ZDIT_ERR_CUDA;
+}
+
+// One cached executable graph of the sampler (zdit_sample_cfg.use_graph).
+struct SampleGraph {
+  std::mutex mu;
+  std::vector<uint8_t> key;
+  cudaGraphExec_t exec = nullptr;
+  int64_t launches = 0;
+  cudaStream_t capture_stream = nullptr;
+  int capture_device = -1;
+};
+
+SampleGraph& sample_graph() {
+  static SampleGraph* g = new SampleGraph();  // never destroyed: outlives the CUDA context at exit
+  return *g;
+}
+
+}  // namespace
+}  // namespace zdit
+
+extern "C" {
+
 ZDIT_API size_t zdit_sample_workspace_bytes(const zdit_stack_cfg* cfg, const zdit_stack_inputs* in) {
   float t_host[kMaxBatch];
   zdit_stack_inputs in2;
@@ -581,29 +637,64 @@ ZDIT_API zdit_status zdit_sample(const zdit_stack_cfg* cfg, const zdit_stack_wei
   Carver c0(nullptr);
   if (workspace_bytes < carve_sample(c0, nullptr, nullptr, nullptr, d)) return ZDIT_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  Carver c(workspace);
-  StackWs ws;
-  float *z = nullptr, *vel = nullptr;
-  carve_sample(c, &ws, &z, &vel, d);
-  in2.patches = z;
-  const int C = d.patch_dim / 4;
-  const int64_t n = (int64_t)d.n_img * d.patch_dim;
-  launch_patchify(latent, z, C, in->grid_h, in->grid_w, 0, s);
-  StackOpts opts;
-  opts.dedup_noise = sc->dedup_noise != 0 && d.B > 1;
-  for (int i = 0; i < sc->n_steps; ++i) {
-    // sigma_i = 3(1-u)/(3(1-u)+u), u = i / n_steps; the DiT sees t = 1 - sigma_i
-    const double u0 = (double)i / sc->n_steps, u1 = (double)(i + 1) / sc->n_steps;
-    const float s0 = (float)(3.0 * (1.0 - u0) / (3.0 * (1.0 - u0) + u0));
-    const float s1 = (float)(3.0 * (1.0 - u1) / (3.0 * (1.0 - u1) + u1));
-    for (int b = 0; b < d.B; ++b) t_host[b] = 1.0f - s0;
-    opts.context_ready = sc->cache_context != 0 && i > 0;
-    zdit_status st = stack_run(cfg, w, &in2, d, ws, vel, opts, s);
-    if (st != ZDIT_OK) return st;
-    launch_euler_cfg(z, vel, d.B > 1 ? vel + n : nullptr, n, sc->guidance, s1 - s0, s);
+  if (!sc->use_graph || profiling_on()) return sample_run(cfg, w, in, sc, latent, workspace, d, in2, t_host, s);
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cap) != cudaSuccess) return ZDIT_ERR_CUDA;
+  if (cap != cudaStreamCaptureStatusNone)  // the caller is capturing: just add our launches
+    return sample_run(cfg, w, in, sc, latent, workspace, d, in2, t_host, s);
+  // key: every argument that shapes the launch sequence
+  std::vector<uint8_t> key;
+  auto put = [&key](const void* p, size_t n) {
+    const uint8_t* b = static_cast<const uint8_t*>(p);
+    key.insert(key.end(), b, b + n);
+  };
+  int dev = 0;
+  cudaGetDevice(&dev);
+  put(&dev, sizeof(dev));
+  put(cfg, sizeof(*cfg));
+  put(w, sizeof(*w));
+  put(w->blocks, sizeof(zdit_block_weights) * (size_t)(cfg->n_noise_refiner + cfg->n_context_refiner + cfg->n_main));
+  put(&in->batch, sizeof(in->batch));
+  put(&in->grid_h, sizeof(in->grid_h));
+  put(&in->grid_w, sizeof(in->grid_w));
+  put(in->n_cap, sizeof(int32_t) * (size_t)in->batch);
+  put(in->n_valid, sizeof(int32_t) * (size_t)in->batch);
+  put(&in->cap_feats, sizeof(in->cap_feats));
+  put(sc, sizeof(*sc));
+  put(&latent, sizeof(latent));
+  put(&workspace, sizeof(workspace));
+  put(&workspace_bytes, sizeof(workspace_bytes));
+  SampleGraph& g = sample_graph();
+  std::lock_guard<std::mutex> lock(g.mu);
+  if (g.exec == nullptr || g.key != key) {
+    // capture on a private stream (the caller's may be the legacy default stream, which
+    // cannot capture); nothing runs during capture, the graph is then launched on `s`
+    if (g.capture_stream == nullptr || g.capture_device != dev) {
+      if (cudaStreamCreateWithFlags(&g.capture_stream, cudaStreamNonBlocking) != cudaSuccess) return ZDIT_ERR_CUDA;
+      g.capture_device = dev;
+    }
+    cudaStream_t cs = g.capture_stream;
+    const int64_t before = zdit_launch_count();
+    if (cudaStreamBeginCapture(cs, cudaStreamCaptureModeRelaxed) != cudaSuccess) return ZDIT_ERR_CUDA;
+    const zdit_status st = sample_run(cfg, w, in, sc, latent, workspace, d, in2, t_host, cs);
+    cudaGraph_t graph = nullptr;
+    const cudaError_t ce = cudaStreamEndCapture(cs, &graph);
+    if (st != ZDIT_OK || ce != cudaSuccess || graph == nullptr) {
+      if (graph != nullptr) cudaGraphDestroy(graph);
+      return st != ZDIT_OK ? st : ZDIT_ERR_CUDA;
+    }
+    cudaGraphExec_t exec = nullptr;
+    const cudaError_t ie = cudaGraphInstantiate(&exec, graph, 0);
+    cudaGraphDestroy(graph);
+    if (ie != cudaSuccess) return ZDIT_ERR_CUDA;
+    if (g.exec != nullptr) cudaGraphExecDestroy(g.exec);
+    g.exec = exec;
+    g.key = key;
+    g.launches = zdit_launch_count() - before;  // counted once at capture, once per replay below
+    return cudaGraphLaunch(g.exec, s) == cudaSuccess ? ZDIT_OK : ZDIT_ERR_CUDA;
   }
-  launch_patchify(z, latent, C, in->grid_h, in->grid_w, 1, s);
-  return cudaGetLastError() == cudaSuccess ? ZDIT_OK : ZDIT_ERR_CUDA;
+  add_launches(g.launches);
+  return cudaGraphLaunch(g.exec, s) == cudaSuccess ? ZDIT_OK : ZDIT_ERR_CUDA;
 }
 
 ZDIT_API zdit_status zdit_euler_cfg_step(float* x, const float* v_pos, const float* v_neg, int64_t n, float g,

@@ -113,6 +113,10 @@ void launch_residual(const ResidArgs& a, cudaStream_t s);
 
 
 int num_sms();
+// true while zdit_profile_begin .. zdit_profile_end is recording
+bool profiling_on();
+// adds n to the launch counter (kernels replayed from a captured graph)
+void add_launches(int64_t n);
 
 // Device address of the library's latched device-error word on the current device.
 int* device_error_ptr();

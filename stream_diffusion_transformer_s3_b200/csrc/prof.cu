@@ -68,6 +68,14 @@ ProfScope::~ProfScope() {
   p.recs.push_back(Rec{kind_, flops_, bytes_, a_, b_});
 }
 
+bool profiling_on() {
+  Prof& p = prof();
+  std::lock_guard<std::mutex> g(p.mu);
+  return p.on;
+}
+
+void add_launches(int64_t n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
 }  // namespace zdit
 
 using namespace zdit;

@@ -30,7 +30,7 @@ def test_library_exports_every_declared_symbol():
 
 def test_version_and_status_strings():
     L = Z.lib()
-    assert L.zdit_version() == 100
+    assert L.zdit_version() == 200
     for code, name in Z.STATUS.items():
         assert L.zdit_status_string(code).decode() == name
 

@@ -102,3 +102,31 @@ def test_sample_caching_is_bitwise_neutral():
     Z.zdit_sample(stack, call, b, ws, cache_context=False)
     assert Z.zdit_device_status() == 0
     assert torch.equal(a, b)
+
+
+def test_sample_as_cuda_graph_is_bitwise_equal():
+    # capture on the first call, replay on later ones; the replay reads the latent's new
+    # contents through the same pointer
+    d, W, latent, caps = _small_setup()
+    stack = Z.DeviceStack(W, dims_of(d), 2, 2, 2, patch_dim=64, cap_dim=128)
+    call = Z.StackCall((8, 8), [64, 32], [45, 1], [0.0, 0.0], dev(caps), dev(caps))
+    ws = torch.empty(Z.sample_workspace_bytes(stack, call), dtype=torch.uint8, device="cuda")
+    plain = dev(latent)
+    Z.zdit_sample(stack, call, plain, ws, n_steps=8, guidance=1.0)
+    lat = dev(latent)
+    n0 = Z.zdit_launch_count()
+    Z.zdit_sample(stack, call, lat, ws, n_steps=8, guidance=1.0, use_graph=True)    # capture + launch
+    n1 = Z.zdit_launch_count()
+    assert Z.zdit_device_status() == 0
+    assert torch.equal(lat, plain)
+    lat.copy_(dev(latent))
+    Z.zdit_sample(stack, call, lat, ws, n_steps=8, guidance=1.0, use_graph=True)    # replay
+    assert Z.zdit_device_status() == 0
+    assert torch.equal(lat, plain)
+    assert Z.zdit_launch_count() - n1 == n1 - n0 > 0
+    other = dev(synth.latent_noise(43, (16, 16, 16)))
+    ref_other = other.clone()
+    Z.zdit_sample(stack, call, ref_other, ws, n_steps=8, guidance=1.0)
+    lat.copy_(other)
+    Z.zdit_sample(stack, call, lat, ws, n_steps=8, guidance=1.0, use_graph=True)    # replay, new noise
+    assert torch.equal(lat, ref_other)
