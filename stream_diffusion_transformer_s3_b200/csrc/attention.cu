@@ -137,6 +137,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int head = blockIdx.y;
+  griddep_wait();     // Q, K, V of the predecessor are complete
+  griddep_trigger();  // every CTA has started: the successor may launch
 
   // locate (branch, query-tile pair) of this CTA
   int b = 0, pair = blockIdx.x;
@@ -443,7 +445,7 @@ zdit_status launch_attention(const AttnArgs& a, cudaStream_t s) {
   }
   ProfScope ps(PROF_ATTENTION, 4.0 * HD * a.n_heads * l2, 4.0 * 2.0 * a.T * (double)cols, s);
   dim3 grid(total_pairs, a.n_heads);
-  attn_tc_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(tq, tk, tv, p);
+  launch_dependent(attn_tc_kernel, grid, dim3(THREADS), SMEM_BYTES, s, tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? ZDIT_OK : ZDIT_ERR_CUDA;
 }
 

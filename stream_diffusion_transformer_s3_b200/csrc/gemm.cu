@@ -276,6 +276,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int num_tiles = p.num_m * p.num_n;
+  griddep_wait();     // the predecessor's output (this GEMM's A operand) is complete
+  griddep_trigger();  // every CTA has started: the successor may launch and set itself up
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -431,6 +433,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int num_tiles = p.num_m * p.num_n;  // num_m counts 256-row pair tiles
+  griddep_wait();     // the predecessor's output (this GEMM's A operand) is complete
+  griddep_trigger();  // every CTA has started: the successor may launch and set itself up
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
@@ -558,7 +562,7 @@ zdit_status launch_epi(const CUtensorMap& ta, const CUtensorMap& tb, const KPara
         return ZDIT_ERR_CUDA;
       attr_pair_set = true;
     }
-    gemm_pair_kernel<EPI><<<grid, THREADS, P_SMEM_BYTES, s>>>(ta, tb, kp);
+    launch_dependent(gemm_pair_kernel<EPI>, dim3(grid), dim3(THREADS), P_SMEM_BYTES, s, ta, tb, kp);
   } else {
     if (!attr_set) {
       if (cudaFuncSetAttribute(gemm_tc_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
@@ -566,7 +570,7 @@ zdit_status launch_epi(const CUtensorMap& ta, const CUtensorMap& tb, const KPara
         return ZDIT_ERR_CUDA;
       attr_set = true;
     }
-    gemm_tc_kernel<EPI><<<grid, THREADS, SMEM_BYTES, s>>>(ta, tb, kp);
+    launch_dependent(gemm_tc_kernel<EPI>, dim3(grid), dim3(THREADS), SMEM_BYTES, s, ta, tb, kp);
   }
   return cudaGetLastError() == cudaSuccess ? ZDIT_OK : ZDIT_ERR_CUDA;
 }

@@ -121,4 +121,32 @@ void add_launches(int64_t n);
 // Device address of the library's latched device-error word on the current device.
 int* device_error_ptr();
 
+// ---------------------------------------------------------------- dependent launches
+// The per-block chain (GEMMs, attention, residual and norm kernels) is launched with
+// programmatic stream serialization: each of these kernels lets its successor launch
+// once all its CTAs have started (griddep_trigger after its prologue), and waits for its
+// predecessor's completion and memory (griddep_wait) before its first global access, so a
+// successor's launch, barrier setup, TMEM allocation and descriptor prefetch overlap the
+// predecessor's last wave.  ZDIT_PDL=0 in the environment turns it off.
+bool pdl_enabled();
+
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                             Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 }  // namespace zdit

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -75,6 +76,18 @@ bool profiling_on() {
 }
 
 void add_launches(int64_t n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+#ifndef ZDIT_PDL_DEFAULT
+#define ZDIT_PDL_DEFAULT 1
+#endif
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("ZDIT_PDL");
+    return e != nullptr ? e[0] != '0' : ZDIT_PDL_DEFAULT != 0;
+  }();
+  return on;
+}
 
 }  // namespace zdit
 

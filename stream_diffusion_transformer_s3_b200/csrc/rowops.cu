@@ -98,6 +98,8 @@ struct NormModParams {
 template <int MAXV>
 __global__ void __launch_bounds__(RT) norm_modulate_kernel(NormModParams p) {
   __shared__ float sh[RT / 32];
+  griddep_wait();
+  griddep_trigger();
   const int t = blockIdx.x;
   const float* xr = p.x + (size_t)t * p.D;
   float4 v[MAXV];
@@ -161,6 +163,8 @@ struct ResidParams {
 template <int MAXV>
 __global__ void __launch_bounds__(RT) residual_kernel(ResidParams p) {
   __shared__ float sh[RT / 32];
+  griddep_wait();
+  griddep_trigger();
   const int t = blockIdx.x;
   const __nv_bfloat16* yr = p.y + (size_t)t * p.D;
   float* xr = p.x + (size_t)t * p.D;
@@ -488,13 +492,13 @@ void launch_norm_modulate_ex(const float* x, int T, int D, const float* w, const
   const int v = (D + RT * 4 - 1) / (RT * 4);
   if (T <= 0) return;
   if (v <= 1)
-    norm_modulate_kernel<1><<<T, RT, 0, s>>>(p);
+    launch_dependent(norm_modulate_kernel<1>, dim3(T), dim3(RT), 0, s, p);
   else if (v <= 2)
-    norm_modulate_kernel<2><<<T, RT, 0, s>>>(p);
+    launch_dependent(norm_modulate_kernel<2>, dim3(T), dim3(RT), 0, s, p);
   else if (v <= 4)
-    norm_modulate_kernel<4><<<T, RT, 0, s>>>(p);
+    launch_dependent(norm_modulate_kernel<4>, dim3(T), dim3(RT), 0, s, p);
   else
-    norm_modulate_kernel<8><<<T, RT, 0, s>>>(p);
+    launch_dependent(norm_modulate_kernel<8>, dim3(T), dim3(RT), 0, s, p);
 }
 
 void launch_norm_modulate(const RowModArgs& a, cudaStream_t s) {
@@ -508,13 +512,13 @@ void launch_residual(const ResidArgs& a, cudaStream_t s) {
   const int v = (a.D + RT * 4 - 1) / (RT * 4);
   if (a.T <= 0) return;
   if (v <= 1)
-    residual_kernel<1><<<a.T, RT, 0, s>>>(p);
+    launch_dependent(residual_kernel<1>, dim3(a.T), dim3(RT), 0, s, p);
   else if (v <= 2)
-    residual_kernel<2><<<a.T, RT, 0, s>>>(p);
+    launch_dependent(residual_kernel<2>, dim3(a.T), dim3(RT), 0, s, p);
   else if (v <= 4)
-    residual_kernel<4><<<a.T, RT, 0, s>>>(p);
+    launch_dependent(residual_kernel<4>, dim3(a.T), dim3(RT), 0, s, p);
   else
-    residual_kernel<8><<<a.T, RT, 0, s>>>(p);
+    launch_dependent(residual_kernel<8>, dim3(a.T), dim3(RT), 0, s, p);
 }
 
 void launch_gemv(const __nv_bfloat16* W, const float* bias, const float* temb, int B, int E, int rows, float* out,

@@ -130,3 +130,21 @@ def test_sample_as_cuda_graph_is_bitwise_equal():
     lat.copy_(other)
     Z.zdit_sample(stack, call, lat, ws, n_steps=8, guidance=1.0, use_graph=True)    # replay, new noise
     assert torch.equal(lat, ref_other)
+
+
+def test_base_recipe_fifty_steps_cfg_four():
+    # the Base-model recipe ([Jobs] "Recipes and precision"): 50 steps, guidance 4, on the
+    # same kernels; the schedule is the same closed form with u = i / 50
+    d, W, latent, caps = _small_setup()
+    stack = Z.DeviceStack(W, dims_of(d), 2, 2, 2, patch_dim=64, cap_dim=128)
+    call = Z.StackCall((8, 8), [64, 32], [45, 1], [0.0, 0.0], dev(caps), dev(caps))
+    ws = torch.empty(Z.sample_workspace_bytes(stack, call), dtype=torch.uint8, device="cuda")
+    lat = dev(latent)
+    Z.zdit_sample(stack, call, lat, ws, n_steps=50, guidance=4.0)
+    assert Z.zdit_device_status() == 0
+    cond = {"caps": caps[:45], "n_cap": 64, "n_valid": 45}
+    unc = {"caps": caps[45:], "n_cap": 32, "n_valid": 1}
+    ref = O.sample(latent, cond, unc, W, d, g=4.0, n_steps=50)
+    e = errors(host(lat), ref)
+    print("\nbase recipe", e)
+    assert e["rel_l2"] <= 2e-2, e
