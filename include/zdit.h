@@ -79,7 +79,7 @@ enum {
  * ffn_hidden % 128 == 0, temb_dim % 8 == 0 and <= 1024,
  * rope_axes[0] + rope_axes[1] + rope_axes[2] == head_dim with every entry even. */
 typedef struct {
-  int32_t dim;          /* D, model width (3840)                           */
+  int32_t dim;          /* D, model width (3840); n_heads * 128, <= 8192    */
   int32_t n_heads;      /* H (30)                                          */
   int32_t head_dim;     /* 128                                             */
   int32_t ffn_hidden;   /* F, SwiGLU hidden width (10240)                  */
@@ -193,7 +193,7 @@ typedef struct {
   int32_t n_context_refiner; /* 2: no-adaLN blocks over the caption tokens only */
   int32_t n_main;            /* 30: blocks over the joint sequence              */
   int32_t patch_dim;         /* 64 = 4 * latent channels                        */
-  int32_t cap_dim;           /* caption feature width (2560)                    */
+  int32_t cap_dim;           /* caption feature width (2560), <= 8192           */
   float t_scale;             /* timestep scale inside the sinusoid (1000)       */
   float final_eps;           /* final LayerNorm epsilon (1e-6)                  */
 } zdit_stack_cfg;

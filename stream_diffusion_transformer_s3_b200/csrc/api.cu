@@ -81,7 +81,9 @@ struct Carver {
 
 bool cfg_ok(const zdit_block_cfg* c) {
   if (c == nullptr) return false;
-  if (c->head_dim != 128 || c->n_heads <= 0 || c->dim != c->n_heads * 128 || c->dim % 256) return false;
+  // dim <= 8192: the row kernels hold a whole row in one CTA's registers
+  if (c->head_dim != 128 || c->n_heads <= 0 || c->dim != c->n_heads * 128 || c->dim % 256 || c->dim > 8192)
+    return false;
   if (c->ffn_hidden <= 0 || c->ffn_hidden % 128) return false;
   if (c->temb_dim <= 0 || c->temb_dim % 8 || c->temb_dim > 1024) return false;
   if (c->rope_axes[0] + c->rope_axes[1] + c->rope_axes[2] != c->head_dim) return false;
@@ -253,7 +255,8 @@ bool stack_dims(const zdit_stack_cfg* cfg, const zdit_stack_inputs* in, StackDim
   if (!in->n_cap || !in->n_valid) return false;
   if (cfg->n_noise_refiner < 0 || cfg->n_context_refiner < 0 || cfg->n_main < 0) return false;
   if (cfg->n_noise_refiner + cfg->n_context_refiner + cfg->n_main > kMaxBlocks) return false;
-  if (cfg->patch_dim <= 0 || cfg->patch_dim % 64 || cfg->cap_dim <= 0 || cfg->cap_dim % 64) return false;
+  if (cfg->patch_dim <= 0 || cfg->patch_dim % 64 || cfg->cap_dim <= 0 || cfg->cap_dim % 64 || cfg->cap_dim > 8192)
+    return false;
   d->B = in->batch;
   d->n_img = in->grid_h * in->grid_w;
   if (d->n_img % 32) return false;

@@ -79,6 +79,8 @@ def test_block_forward_rejects_bad_arguments_before_launch():
     bad2 = d.cfg(Z.flags_of())
     bad2.rope_axes[0] = 30
     assert call(args(cfg=C.byref(bad2))) == -2
+    wide = Z.Dims(dim=8448, n_heads=66, ffn_hidden=768).cfg(Z.flags_of())  # rows wider than 8192
+    assert call(args(cfg=C.byref(wide))) == -2
     cu_bad = (C.c_int32 * 3)(0, 50, 40)
     vl_bad = Z.Varlen(2, _fake(), cu_bad)
     assert call(args(vl=C.byref(vl_bad))) == -2
@@ -106,6 +108,8 @@ def test_stack_dims_validation():
     assert L.zdit_stack_workspace_bytes(C.byref(cfg), C.byref(bad)) == 0
     odd_grid = Z.StackInputs(2, 5, 5, n_cap, n_val, _fake(), _fake(), t)   # 25 image tokens
     assert L.zdit_stack_workspace_bytes(C.byref(cfg), C.byref(odd_grid)) == 0
+    wide_cap = Z.StackCfg(d.cfg(Z.flags_of()), 2, 2, 2, 64, 8256, 1000.0, 1e-6)  # caption width > 8192
+    assert L.zdit_stack_workspace_bytes(C.byref(wide_cap), C.byref(ok)) == 0
 
 
 def test_euler_rejects_null_and_misaligned():
