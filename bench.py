@@ -140,6 +140,44 @@ BLOCK_WORKLOAD = ("one main DiT block of the 1024x1024 workload: joint cond/unco
                   "tokens, width 3840, 30x128 heads, SwiGLU 10240, adaLN + sandwich norm")
 
 
+ATTN_SWEEP_IMG = (1024, 4096, 9216, 16384)
+ATTN_SWEEP_CAP = (32, 128, 512)   # cond caption length; uncond 32
+ATTN_SWEEP_LARGEST = (16384, (512, 32))
+ATTN_WORKLOAD = ("joint attention alone: cond/uncond branches of 16384 image tokens + captions 512 / 32, "
+                 "30 x 128 heads, Q/K/V N(0,1) bf16; sweep over image tokens {1024, 4096, 9216, 16384} x "
+                 "cond caption {32, 128, 512}")
+
+
+def attention_sweep(torch, Z, device, reps=5):
+    """TFLOP/s of zdit_joint_attention over the image-token x caption-length grid (CUDA
+    events, median of `reps` launches after 2 warm-up launches)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(7)
+    out = {}
+    for n_i in ATTN_SWEEP_IMG:
+        for c in ATTN_SWEEP_CAP:
+            lens = [n_i + c, n_i + 32]
+            vl = Z.DeviceVarlen([0, lens[0], lens[0] + lens[1]], device=device)
+            T = vl.total
+            q, k, v = (torch.randn(T, H * HD, generator=g).to(device=device, dtype=torch.bfloat16)
+                       for _ in range(3))
+            o = torch.empty(T, H * HD, device=device, dtype=torch.bfloat16)
+            for _ in range(2):
+                Z.zdit_joint_attention(q, k, v, o, vl, H)
+            times = []
+            for _ in range(reps):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                Z.zdit_joint_attention(q, k, v, o, vl, H)
+                e1.record()
+                torch.cuda.synchronize()
+                times.append(e0.elapsed_time(e1))
+            ms = statistics.median(times)
+            out[f"{n_i}+{c}/{n_i}+32"] = round(sum(4.0 * D * L * L for L in lens) / (ms * 1e-3) / 1e12, 1)
+            del q, k, v, o
+    return out
+
+
 def build_block(torch, Z, device, seed=99):
     g = torch.Generator(device=device)
     g.manual_seed(seed)
@@ -210,6 +248,20 @@ def run_ours(args):
             call.set_t([1.0 - s0, 1.0 - s0])
             Z.zdit_stack_forward(stack, call, out, ws)
             Z.zdit_euler_cfg_step(z, out[0], out[1], 1.0, s0, s1)
+    elif args.workload == "attention":
+        # joint attention alone at the largest size of the sweep: 16384 image tokens, caption
+        # 512 (cond) / 32 (uncond), 30 heads x 128; Q, K, V N(0, 1) in bf16 (after RoPE)
+        n_i, caps_ = ATTN_SWEEP_LARGEST
+        lens = [n_i + caps_[0], n_i + caps_[1]]
+        vl = Z.DeviceVarlen([0, lens[0], lens[0] + lens[1]], device=device)
+        T = vl.total
+        q, k, v = (torch.randn(T, H * HD, generator=g).to(device=device, dtype=torch.bfloat16) for _ in range(3))
+        o = torch.empty(T, H * HD, device=device, dtype=torch.bfloat16)
+        inputs, result = [q, k, v], o
+        flops = sum(4.0 * D * L * L for L in lens)
+
+        def step(i):
+            Z.zdit_joint_attention(q, k, v, o, vl, H)
     elif args.workload == "sampler":
         # one 1024x1024 image: 8 sampler steps on the cond/uncond pair in one call
         stack = build_model(torch, Z, device)
@@ -343,7 +395,7 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": {"stack": WORKLOAD, "block": BLOCK_WORKLOAD,
-                                    "sampler": SAMPLER_WORKLOAD}[args.workload],
+                                    "sampler": SAMPLER_WORKLOAD, "attention": ATTN_WORKLOAD}[args.workload],
                        "global_batch": 2 * world, "seq_len": [n_img + c for c in N_CAPS],
                        "flops_per_forward": flops, "parallelism": f"replicas x{world}",
                        "l2": ("working set larger than L2 (12.3 GB of bf16 weights streamed per step)" if args.workload == "stack" else "working set larger than L2 (354 MB weights + 128 MB residual + 448 MB activations per block)"),
@@ -358,6 +410,11 @@ def run_ours(args):
         }
         if args.workload == "block":
             res["metric"] = "DiT main-block forward TFLOP/s (1024^2 cond/uncond sequence, bf16, 1 B200)"
+        if args.workload == "attention":
+            res["metric"] = "joint attention TFLOP/s (30 x 128 heads, cond/uncond branches, bf16, 1 B200)"
+            res["config"]["seq_len"] = [ATTN_SWEEP_LARGEST[0] + c for c in ATTN_SWEEP_LARGEST[1]]
+            res["config"]["l2"] = "Q, K, V and O (1 GB) larger than L2"
+            res["sweep"] = attention_sweep(torch, Z, device)
         if args.workload == "sampler":
             res["metric"] = "s per 1024^2 image, 8-step negated-CFG sampler (bf16, 1 B200)"
             res["value"] = round(ms / 1e3, 4)
@@ -371,7 +428,8 @@ def run_ours(args):
                                                              if args.dedup else "")
                                          + (", captured as one CUDA graph and replayed" if args.graph else ""))
         if world == 1 and not args.no_cpu_baseline:
-            res["cpu_baseline"] = cpu_baseline_block(seconds=None)
+            res["cpu_baseline"] = (cpu_baseline_attention() if args.workload == "attention"
+                                   else cpu_baseline_block(seconds=None))
         print(json.dumps(res), flush=True)
     if world > 1:
         dist.destroy_process_group()
@@ -411,6 +469,22 @@ def cpu_baseline_block(seconds=None):
                       f"NumPy float64 oracle, {dt:.1f} s"}
 
 
+def cpu_baseline_attention():
+    """The oracle's joint attention on a bounded sample of the attention workload: one head
+    of the cond branch at 4096 + 512 tokens."""
+    import numpy as np
+    import oracle as O
+    from stream_diffusion_transformer_s3_b200 import synth
+    L = 4096 + 512
+    q, k, v = (synth.bf16_round(synth.randn(11, i, (L, HD))).astype(np.float64) for i in range(3))
+    t0 = time.perf_counter()
+    O.softmax_attention(q, k, v)
+    dt = time.perf_counter() - t0
+    return {"value": round(4.0 * HD * L * L / dt / 1e12, 5), "unit": "TFLOP/s", "cores": _cores(),
+            "kind": "oracle", "sample": f"one head of the cond branch at 4096 + 512 tokens, NumPy float64 "
+                                        f"oracle, {dt:.1f} s"}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -446,9 +520,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["stack", "block", "sampler"], default="stack",
+    ap.add_argument("--workload", choices=["stack", "block", "sampler", "attention"], default="stack",
                     help="stack: the full DiT step (default); block: one main block (for kernel captures); "
-                         "sampler: one whole 8-step image per step")
+                         "sampler: one whole 8-step image per step; attention: joint attention alone at "
+                         "16384 image tokens, with a sweep over sequence lengths")
     ap.add_argument("--graph", action="store_true",
                     help="sampler workload: the whole image as one captured CUDA graph, replayed")
     ap.add_argument("--dedup", action="store_true",
