@@ -148,9 +148,9 @@ ATTN_WORKLOAD = ("joint attention alone: cond/uncond branches of 16384 image tok
                  "cond caption {32, 128, 512}")
 
 
-def attention_sweep(torch, Z, device, reps=5):
+def attention_sweep(torch, Z, device, reps=3, per=10):
     """TFLOP/s of zdit_joint_attention over the image-token x caption-length grid (CUDA
-    events, median of `reps` launches after 2 warm-up launches)."""
+    events around `per` back-to-back launches, median of `reps`, after 2 warm-up launches)."""
     g = torch.Generator(device="cpu")
     g.manual_seed(7)
     out = {}
@@ -168,10 +168,11 @@ def attention_sweep(torch, Z, device, reps=5):
             for _ in range(reps):
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record()
-                Z.zdit_joint_attention(q, k, v, o, vl, H)
+                for _ in range(per):
+                    Z.zdit_joint_attention(q, k, v, o, vl, H)
                 e1.record()
                 torch.cuda.synchronize()
-                times.append(e0.elapsed_time(e1))
+                times.append(e0.elapsed_time(e1) / per)
             ms = statistics.median(times)
             out[f"{n_i}+{c}/{n_i}+32"] = round(sum(4.0 * D * L * L for L in lens) / (ms * 1e-3) / 1e12, 1)
             del q, k, v, o
