@@ -47,9 +47,6 @@ constexpr int OFF_V = OFF_K + 2 * TILE_BYTES;
 constexpr int OFF_BAR = OFF_V + 2 * TILE_BYTES;
 constexpr int SMEM_BYTES = 1024 + OFF_BAR + 256;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-// Of every 4 pairs of exponentials, how many run on the FMA pipe (exp2_poly2)
-// instead of MUFU.  Measured on B200: MUFU is not the limit of this kernel, so 0.
-constexpr int kPolyPairsPer4 = 0;
 
 struct AParams {
   int ldo, n_heads, batch;
@@ -89,31 +86,6 @@ __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
   uint64_t r;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
-}
-
-// 2^x for a pair, on the FMA/ALU pipes instead of MUFU, for x <= 8 (x may be -inf).
-// x is clamped to -125 (below that the result is 0), split as x = n + f with n = round(x) (the 1.5 * 2^23 shift
-// trick) and f in [-1/2, 1/2]; 2^f is a cubic fitted in relative error on that
-// interval by least squares (max relative error 2.2e-4, far below the bf16
-// rounding of P); 2^n is added into the exponent field.
-__device__ __forceinline__ void exp2_poly2(uint64_t x2, float& y0, float& y1) {
-  float a0, b0;
-  unpk2(x2, a0, b0);
-  const float a = fmaxf(a0, -125.f), b = fmaxf(b0, -125.f);  // keeps 2^n a normal number
-  const uint64_t shift = pk2(12582912.0f, 12582912.0f);
-  const uint64_t nshift = pk2(-12582912.0f, -12582912.0f);
-  const uint64_t xc = pk2(a, b);
-  const uint64_t t = add2(xc, shift);              // round(x) in the low mantissa bits
-  const uint64_t f = add2(xc, add2(t, nshift) ^ 0x8000000080000000ull);  // x - round(x)
-  uint64_t q = pk2(5.286743492e-02f, 5.286743492e-02f);
-  q = fma2(q, f, pk2(2.421518862e-01f, 2.421518862e-01f));
-  q = fma2(q, f, pk2(6.935867667e-01f, 6.935867667e-01f));
-  q = fma2(q, f, pk2(9.999627471e-01f, 9.999627471e-01f));
-  float q0, q1, t0, t1;
-  unpk2(q, q0, q1);
-  unpk2(t, t0, t1);
-  y0 = a0 < -125.f ? 0.f : __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
-  y1 = b0 < -125.f ? 0.f : __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 
 __global__ void __launch_bounds__(THREADS, 1)
@@ -336,9 +308,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           tmem_st16(tO + c * 16, r);
         }
       }
-      // P = exp2(s * scale - m_ref), packed bf16 pairs over the first 64 columns of S_t
-      // P = exp2(s * scale - m_ref) with packed f32x2 arithmetic (optionally a share
-      // of the exponentials on the FMA pipe, kPolyPairsPer4).
+      // P = exp2(s * scale - m_ref) with packed f32x2 arithmetic, bf16 pairs over the
+      // first 64 columns of S_t
       const uint64_t sc2 = pk2(p.scale_log2, p.scale_log2);
       const uint64_t nm2 = pk2(-m_ref, -m_ref);
       uint64_t part[4] = {0ull, 0ull, 0ull, 0ull};  // 4 independent packed sum chains
@@ -348,15 +319,9 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const uint64_t x2 = fma2(pk2(s[c * 32 + 2 * e], s[c * 32 + 2 * e + 1]), sc2, nm2);
-          float p0, p1;
-          if ((e & 3) >= 4 - kPolyPairsPer4) {
-            exp2_poly2(x2, p0, p1);
-          } else {
-            float a, b;
-            unpk2(x2, a, b);
-            p0 = ex2(a);
-            p1 = ex2(b);
-          }
+          float a, b;
+          unpk2(x2, a, b);
+          const float p0 = ex2(a), p1 = ex2(b);
           part[e & 3] = add2(part[e & 3], pk2(p0, p1));
           pk[e] = pack_bf16x2(p0, p1);
         }
