@@ -422,3 +422,60 @@ def test_synth_bf16_rounding_is_nearest_even():
     assert r[0] == 1.0 and r[1] == 1.0 and r[2] == 1.0 + 2 ** -6 and r[3] == -2.5
     np.testing.assert_array_equal(
         r, torch.from_numpy(x).to(torch.bfloat16).to(torch.float32).numpy())
+
+
+def _tiny_stack(seed=5, n_noise=1, n_context=1, n_main=1):
+    d = synth.BlockDims(dim=256, n_heads=2, head_dim=128, ffn_hidden=384)
+    W = synth.stack_weights(seed, d, n_noise=n_noise, n_context=n_context, n_main=n_main, cap_dim=64)
+    case = synth.stack_case(seed, 4, 4, [64, 32], [45, 1], [0.3, 0.7], cap_dim=64)
+    return d, W, case
+
+
+def _zero_projections(wb):
+    wb = dict(wb)
+    for k in ("w_qkv", "w_out", "w1", "w3", "w2"):
+        wb[k] = np.zeros_like(wb[k])
+    return wb
+
+
+def test_stack_with_zero_projections_is_embed_then_final_layer():
+    # every block's projections zero => every block adds exactly 0 to its residual, so the
+    # stack reduces to x-embed of the image rows followed by the final layer; the expected
+    # value is composed here from torch float64 routines (Linear, LayerNorm, SiLU, cos/sin)
+    d, W, case = _tiny_stack()
+    Wz = dict(W, blocks=[_zero_projections(wb) for wb in W["blocks"]])
+    out = O.stack_forward(case, Wz, d)
+    t64 = lambda a: torch.as_tensor(np.asarray(a, np.float64))
+    half = d.temb_dim // 2
+    freqs = torch.exp(-math.log(10000.0) * torch.arange(half, dtype=torch.float64) / half)
+    args = 1000.0 * t64(case["t"])[:, None] * freqs[None, :]
+    emb = torch.cat([torch.cos(args), torch.sin(args)], dim=1)
+    temb = torch.nn.functional.linear(torch.nn.functional.silu(
+        torch.nn.functional.linear(emb, t64(W["w_t1"]), t64(W["b_t1"]))), t64(W["w_t2"]), t64(W["b_t2"]))
+    for b in range(2):
+        x = torch.nn.functional.linear(t64(case["patches"][b]), t64(W["w_x"]), t64(W["b_x"]))
+        scale = torch.nn.functional.linear(temb[b], t64(W["w_fada"]), t64(W["b_fada"]))
+        a = torch.nn.functional.layer_norm(x, (x.shape[-1],), eps=1e-6) * (1.0 + scale)
+        ref = torch.nn.functional.linear(a, t64(W["w_final"]), t64(W["b_final"])).numpy()
+        np.testing.assert_allclose(out[b], ref, rtol=1e-10, atol=1e-10)
+
+
+def test_stack_branch_alone_equals_branch_in_pair():
+    # branches never mix: the cond branch run alone gives the cond output of the pair
+    d, W, case = _tiny_stack(seed=6)
+    pair = O.stack_forward(case, W, d)
+    alone = dict(case, patches=case["patches"][:1], caps=case["caps"][:45], n_caps=[64], n_valids=[45],
+                 t=case["t"][:1])
+    one = O.stack_forward(alone, W, d)
+    np.testing.assert_allclose(one[0], pair[0], rtol=1e-12, atol=1e-12)
+
+
+def test_captions_reach_the_image_only_through_main_blocks():
+    # with the main blocks' projections zero, the image output does not depend on the
+    # caption at all; with them live it does
+    d, W, case = _tiny_stack(seed=8)
+    kinds = W["block_kinds"]
+    Wm = dict(W, blocks=[_zero_projections(wb) if k == "main" else wb for wb, k in zip(W["blocks"], kinds)])
+    other = dict(case, caps=case["caps"] + 0.5)
+    np.testing.assert_allclose(O.stack_forward(other, Wm, d), O.stack_forward(case, Wm, d), rtol=0, atol=0)
+    assert np.abs(O.stack_forward(other, W, d) - O.stack_forward(case, W, d)).max() > 1e-6
