@@ -38,6 +38,13 @@ Readings where the pages are silent (each is also listed in the design notes):
   R8  Caption embed: RMSNorm over the caption width (weighted) then Linear + bias; the
       rows at index >= n_valid are replaced by the learned pad vector.
   R9  QK-norm (per-head RMSNorm of q and k before RoPE) is an option, off by default.
+
+Pins: every function is checked in tests/test_oracle.py against library routines, brute
+force, closed forms, invariants or values printed on the pages.  stack_forward and sample:
+parity unpinned as a whole (the pages print no output value); their parts are pinned, and so
+are stack-level invariants (zero projections reduce the stack to embed + final layer, branch
+isolation, captions acting only through the main blocks) and sampler invariants (schedule,
+telescoping Euler steps, negated CFG cases).
 """
 from __future__ import annotations
 
