@@ -378,16 +378,26 @@ __global__ void timestep_embed_kernel(TembParams tp, int E, float t_scale, const
     emb[e] = (float)(e < half ? cos(arg) : sin(arg));
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    float a = b1[e];
-    for (int k = 0; k < E; ++k) a += __bfloat162float(w1[(size_t)e * E + k]) * emb[k];
-    hid[e] = a / (1.0f + expf(-a));
+  // the two E x E products: a warp per output row, lanes split the row in 16-byte pieces
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  auto row_dot = [&](const __nv_bfloat16* wr, const float* v) {
+    float a = 0.f;
+    for (int k = lane * 8; k < E; k += 256) {
+      const uint4 u = *reinterpret_cast<const uint4*>(wr + k);
+      const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&u);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) a += __bfloat162float(h[j]) * v[k + j];
+    }
+    return warp_sum(a);
+  };
+  for (int e = warp; e < E; e += nw) {
+    const float a = row_dot(w1 + (size_t)e * E, emb) + b1[e];
+    if (lane == 0) hid[e] = a / (1.0f + expf(-a));
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    float a = b2[e];
-    for (int k = 0; k < E; ++k) a += __bfloat162float(w2[(size_t)e * E + k]) * hid[k];
-    temb[(size_t)b * E + e] = a;
+  for (int e = warp; e < E; e += nw) {
+    const float a = row_dot(w2 + (size_t)e * E, hid) + b2[e];
+    if (lane == 0) temb[(size_t)b * E + e] = a;
   }
 }
 
