@@ -10,7 +10,7 @@
 // Warp roles (320 threads):
 //   warps 0-3 : softmax of query tile 0, one thread per query row (TMEM lane)
 //   warps 4-7 : softmax of query tile 1
-//   warp 8    : TMA producer (Q0, Q1 once; K and V tiles in separate 2-deep rings)
+//   warp 8    : TMA producer (Q0, K0, then Q1; K and V tiles in separate 2-deep rings)
 //   warp 9    : tcgen05.mma issuer
 // TMEM columns: S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).  P_t (bf16,
 // two per 32-bit column) is written back over the first 64 columns of S_t and fed
@@ -22,6 +22,8 @@
 // Online softmax in FP32 with a lazily moved reference max: the running max only
 // moves (and O is rescaled) when a row's max grows by more than 2^8, so the common
 // tile needs no O round trip; P = exp2(s - m_ref) <= 256 stays in bf16 range.
+// The epilogue stages O / l as bf16 in the shared memory that Q and the K ring no
+// longer need, then writes two full 256-byte rows per warp store instruction.
 #include <cstdio>
 
 #include "internal.h"
@@ -94,16 +96,16 @@ __global__ void __launch_bounds__(THREADS, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-  uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;    // [2]
-  uint64_t* k_empty = bars + 3;   // [2]
-  uint64_t* v_full = bars + 5;    // [2]
-  uint64_t* v_empty = bars + 7;   // [2]
-  uint64_t* s_full = bars + 9;    // [2] one per query tile
-  uint64_t* p_full = bars + 11;   // [2]
-  uint64_t* o_full = bars + 13;   // [2]
-  uint64_t* mma_done = bars + 15;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* q_full = bars + 0;    // [2] one per query tile
+  uint64_t* k_full = bars + 2;    // [2]
+  uint64_t* k_empty = bars + 4;   // [2]
+  uint64_t* v_full = bars + 6;    // [2]
+  uint64_t* v_empty = bars + 8;   // [2]
+  uint64_t* s_full = bars + 10;   // [2] one per query tile
+  uint64_t* p_full = bars + 12;   // [2]
+  uint64_t* o_full = bars + 14;   // [2]
+  uint64_t* mma_done = bars + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -127,8 +129,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int q0 = seg0 + pair * 2 * TILE;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
     for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
       mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
       mbar_init(&v_full[i], 1);
@@ -155,12 +157,11 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (warp == WARP_LOAD && lane == 0) {
     // ------------------------------------------------------------ producer
+    // Q0, then K0, then Q1: the first S product waits for 64 KB instead of 96 KB
     uint8_t* sQ = smem + OFF_Q;
-    mbar_arrive_expect_tx(q_full, 2 * TILE_BYTES);
-    tma_load_2d(sQ, &tmQ, q_full, col0, q0);
-    tma_load_2d(sQ + HALF, &tmQ, q_full, col0 + 64, q0);
-    tma_load_2d(sQ + TILE_BYTES, &tmQ, q_full, col0, q0 + TILE);
-    tma_load_2d(sQ + TILE_BYTES + HALF, &tmQ, q_full, col0 + 64, q0 + TILE);
+    mbar_arrive_expect_tx(&q_full[0], TILE_BYTES);
+    tma_load_2d(sQ, &tmQ, &q_full[0], col0, q0);
+    tma_load_2d(sQ + HALF, &tmQ, &q_full[0], col0 + 64, q0);
     int nk_issued = 0, nv_issued = 0;
     for (int j = 0; j < n_kv; ++j) {
       const int st = j & 1;
@@ -172,6 +173,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       tma_load_2d(sK, &tmK, &k_full[st], col0, r0);
       tma_load_2d(sK + HALF, &tmK, &k_full[st], col0 + 64, r0);
       ++nk_issued;
+      if (j == 0) {
+        mbar_arrive_expect_tx(&q_full[1], TILE_BYTES);
+        tma_load_2d(sQ + TILE_BYTES, &tmQ, &q_full[1], col0, q0 + TILE);
+        tma_load_2d(sQ + TILE_BYTES + HALF, &tmQ, &q_full[1], col0 + 64, q0 + TILE);
+      }
       if (!mbar_wait(&v_empty[st], par, abort_flag, p.err)) break;
       uint8_t* sV = smem + OFF_V + st * TILE_BYTES;
       mbar_arrive_expect_tx(&v_full[st], TILE_BYTES);
@@ -181,7 +187,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     if (*abort_flag) {
       int dummy = 0;
-      mbar_wait(q_full, 0, &dummy);
+      mbar_wait(&q_full[0], 0, &dummy);
+      if (nk_issued > 0) mbar_wait(&q_full[1], 0, &dummy);
       for (int j = (nk_issued > 2 ? nk_issued - 2 : 0); j < nk_issued; ++j)
         mbar_wait(&k_full[j & 1], (j >> 1) & 1, &dummy);
       for (int j = (nv_issued > 2 ? nv_issued - 2 : 0); j < nv_issued; ++j)
@@ -225,7 +232,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int k = 1; k < HD / 16; ++k) umma_bf16_ss(d, qb + koff(k), kb + koff(k), id_s, 1u);
       umma_commit(&s_full[t]);
     };
-    bool ok = mbar_wait(q_full, 0, abort_flag, p.err);
+    bool ok = mbar_wait(&q_full[0], 0, abort_flag, p.err);
     for (int j = 0; ok && j < n_kv; ++j) {
       if (!mbar_wait(&k_full[j & 1], (j >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
       tc_fence_after();
@@ -235,6 +242,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (!issue_pv(1, j - 1)) { ok = false; break; }
         umma_commit(&v_empty[(j - 1) & 1]);
       }
+      if (j == 0 && !mbar_wait(&q_full[1], 0, abort_flag, p.err)) { ok = false; break; }
       issue_s(1, j);
       umma_commit(&k_empty[j & 1]);
     }
@@ -341,24 +349,36 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_full[t], 0, abort_flag, p.err));
     if (ok) {
       tc_fence_after();
-      const int qrow = pair * 2 * TILE + t * TILE + row;
+      // O_t / l, staged as bf16 in shared memory so the global stores are coalesced: once
+      // O_t is final every S product has completed, so Q and the K ring are idle (tile t
+      // uses the t-th 64 KB; rows padded to 272 B keep the row-per-lane writes
+      // conflict-free).
+      constexpr int kStageRow = 2 * HD + 16;
+      uint8_t* stage = smem + OFF_Q + t * 65536 + lg * 32 * kStageRow;
       const float inv = 1.0f / l_sum;
-      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) + (size_t)(seg0 + qrow) * p.ldo + col0;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t r[32];
-        __syncwarp();
         tmem_ld32(tO + c * 32, r);
         tmem_ld_wait();
-        if (qrow < L) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+        uint4* dst = reinterpret_cast<uint4*>(stage + lane * kStageRow + c * 64);
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            dst[e] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * e]) * inv, __uint_as_float(r[8 * e + 1]) * inv),
-                                pack_bf16x2(__uint_as_float(r[8 * e + 2]) * inv, __uint_as_float(r[8 * e + 3]) * inv),
-                                pack_bf16x2(__uint_as_float(r[8 * e + 4]) * inv, __uint_as_float(r[8 * e + 5]) * inv),
-                                pack_bf16x2(__uint_as_float(r[8 * e + 6]) * inv, __uint_as_float(r[8 * e + 7]) * inv));
-        }
+        for (int e = 0; e < 4; ++e)
+          dst[e] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * e]) * inv, __uint_as_float(r[8 * e + 1]) * inv),
+                              pack_bf16x2(__uint_as_float(r[8 * e + 2]) * inv, __uint_as_float(r[8 * e + 3]) * inv),
+                              pack_bf16x2(__uint_as_float(r[8 * e + 4]) * inv, __uint_as_float(r[8 * e + 5]) * inv),
+                              pack_bf16x2(__uint_as_float(r[8 * e + 6]) * inv, __uint_as_float(r[8 * e + 7]) * inv));
+      }
+      __syncwarp();
+      // two 256-byte rows per warp instruction
+      const int row0 = pair * 2 * TILE + t * TILE + lg * 32;
+#pragma unroll 4
+      for (int it = 0; it < 16; ++it) {
+        const int r = it * 2 + (lane >> 4);
+        const uint4 v = *reinterpret_cast<const uint4*>(stage + r * kStageRow + (lane & 15) * 16);
+        if (row0 + r < L)
+          *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + (size_t)(seg0 + row0 + r) * p.ldo + col0 +
+                                    (lane & 15) * 8) = v;
       }
     }
   }
