@@ -7,11 +7,13 @@
 // branches never see each other, and only the columns past the segment end of the
 // last key tile are excluded.
 //
-// Warp roles (320 threads):
+// Warp roles (384 threads, three warpgroups):
 //   warps 0-3 : softmax of query tile 0, one thread per query row (TMEM lane)
 //   warps 4-7 : softmax of query tile 1
 //   warp 8    : TMA producer (Q0, K0, then Q1; K and V tiles in separate 2-deep rings)
 //   warp 9    : tcgen05.mma issuer
+//   warps 10-11 complete the control warpgroup, which hands registers to the softmax
+//   warpgroups (setmaxnreg: 168 at launch -> 208 softmax, 88 control).
 // TMEM columns: S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).  P_t (bf16,
 // two per 32-bit column) is written back over the first 64 columns of S_t and fed
 // to the PV product straight from TMEM, so P never touches shared memory.
@@ -40,7 +42,7 @@ constexpr int TILE = 128;            // query rows and key rows per tile
 constexpr int HD = 128;              // head dim
 constexpr int HALF = TILE * 64 * 2;  // one 64-column swizzled half tile: 16 KB
 constexpr int TILE_BYTES = 2 * HALF;
-constexpr int THREADS = 320;
+constexpr int THREADS = 384;  // three warpgroups: softmax tile 0, softmax tile 1, control
 constexpr int WARP_LOAD = 8, WARP_MMA = 9;
 // smem: Q0 | Q1 | K[2] | V[2], then barriers
 constexpr int OFF_Q = 0;
@@ -155,108 +157,115 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t tmem = *tmem_slot;
   const int col0 = head * HD;
 
-  if (warp == WARP_LOAD && lane == 0) {
-    // ------------------------------------------------------------ producer
-    // Q0, then K0, then Q1: the first S product waits for 64 KB instead of 96 KB
-    uint8_t* sQ = smem + OFF_Q;
-    mbar_arrive_expect_tx(&q_full[0], TILE_BYTES);
-    tma_load_2d(sQ, &tmQ, &q_full[0], col0, q0);
-    tma_load_2d(sQ + HALF, &tmQ, &q_full[0], col0 + 64, q0);
-    int nk_issued = 0, nv_issued = 0;
-    for (int j = 0; j < n_kv; ++j) {
-      const int st = j & 1;
-      const uint32_t par = ((j >> 1) & 1) ^ 1;
-      const int r0 = seg0 + j * TILE;
-      if (!mbar_wait(&k_empty[st], par, abort_flag, p.err)) break;
-      uint8_t* sK = smem + OFF_K + st * TILE_BYTES;
-      mbar_arrive_expect_tx(&k_full[st], TILE_BYTES);
-      tma_load_2d(sK, &tmK, &k_full[st], col0, r0);
-      tma_load_2d(sK + HALF, &tmK, &k_full[st], col0 + 64, r0);
-      ++nk_issued;
-      if (j == 0) {
-        mbar_arrive_expect_tx(&q_full[1], TILE_BYTES);
-        tma_load_2d(sQ + TILE_BYTES, &tmQ, &q_full[1], col0, q0 + TILE);
-        tma_load_2d(sQ + TILE_BYTES + HALF, &tmQ, &q_full[1], col0 + 64, q0 + TILE);
+  // Register split: launched with 168 per thread (384 x 168 = 64512); the control
+  // warpgroup drops to 88 and the two softmax warpgroups rise to 208:
+  // 2 x 128 x 208 + 128 x 88 = 64512, exactly the launch's registers.
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 88;\n" ::: "memory");
+    if (warp == WARP_LOAD && lane == 0) {
+      // ------------------------------------------------------------ producer
+      // Q0, then K0, then Q1: the first S product waits for 64 KB instead of 96 KB
+      uint8_t* sQ = smem + OFF_Q;
+      mbar_arrive_expect_tx(&q_full[0], TILE_BYTES);
+      tma_load_2d(sQ, &tmQ, &q_full[0], col0, q0);
+      tma_load_2d(sQ + HALF, &tmQ, &q_full[0], col0 + 64, q0);
+      int nk_issued = 0, nv_issued = 0;
+      for (int j = 0; j < n_kv; ++j) {
+        const int st = j & 1;
+        const uint32_t par = ((j >> 1) & 1) ^ 1;
+        const int r0 = seg0 + j * TILE;
+        if (!mbar_wait(&k_empty[st], par, abort_flag, p.err)) break;
+        uint8_t* sK = smem + OFF_K + st * TILE_BYTES;
+        mbar_arrive_expect_tx(&k_full[st], TILE_BYTES);
+        tma_load_2d(sK, &tmK, &k_full[st], col0, r0);
+        tma_load_2d(sK + HALF, &tmK, &k_full[st], col0 + 64, r0);
+        ++nk_issued;
+        if (j == 0) {
+          mbar_arrive_expect_tx(&q_full[1], TILE_BYTES);
+          tma_load_2d(sQ + TILE_BYTES, &tmQ, &q_full[1], col0, q0 + TILE);
+          tma_load_2d(sQ + TILE_BYTES + HALF, &tmQ, &q_full[1], col0 + 64, q0 + TILE);
+        }
+        if (!mbar_wait(&v_empty[st], par, abort_flag, p.err)) break;
+        uint8_t* sV = smem + OFF_V + st * TILE_BYTES;
+        mbar_arrive_expect_tx(&v_full[st], TILE_BYTES);
+        tma_load_2d(sV, &tmV, &v_full[st], col0, r0);
+        tma_load_2d(sV + HALF, &tmV, &v_full[st], col0 + 64, r0);
+        ++nv_issued;
       }
-      if (!mbar_wait(&v_empty[st], par, abort_flag, p.err)) break;
-      uint8_t* sV = smem + OFF_V + st * TILE_BYTES;
-      mbar_arrive_expect_tx(&v_full[st], TILE_BYTES);
-      tma_load_2d(sV, &tmV, &v_full[st], col0, r0);
-      tma_load_2d(sV + HALF, &tmV, &v_full[st], col0 + 64, r0);
-      ++nv_issued;
-    }
-    if (*abort_flag) {
+      if (*abort_flag) {
+        int dummy = 0;
+        mbar_wait(&q_full[0], 0, &dummy);
+        if (nk_issued > 0) mbar_wait(&q_full[1], 0, &dummy);
+        for (int j = (nk_issued > 2 ? nk_issued - 2 : 0); j < nk_issued; ++j)
+          mbar_wait(&k_full[j & 1], (j >> 1) & 1, &dummy);
+        for (int j = (nv_issued > 2 ? nv_issued - 2 : 0); j < nv_issued; ++j)
+          mbar_wait(&v_full[j & 1], (j >> 1) & 1, &dummy);
+      }
+    } else if (warp == WARP_MMA && lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      // Each UMMA here is only 64 tensor clocks of work, so the issuing thread must do
+      // almost nothing per instruction: every shared-memory descriptor is precomputed
+      // (a descriptor is linear in the address: desc(addr + off) = desc(addr) + off / 16).
+      const uint32_t id_s = idesc_bf16_f32(TILE, TILE);             // Q, K both K-major
+      const uint32_t id_o = idesc_bf16_f32(TILE, HD, false, true);  // P from TMEM, V MN-major
+      uint64_t dq[2], dk[2], dv[2];
+      for (int t = 0; t < 2; ++t) dq[t] = sdesc_kmajor_sw128(smem_u32(smem + OFF_Q + t * TILE_BYTES));
+      for (int i = 0; i < 2; ++i) dk[i] = sdesc_kmajor_sw128(smem_u32(smem + OFF_K + i * TILE_BYTES));
+      for (int i = 0; i < 2; ++i) dv[i] = sdesc_mnmajor_sw128(smem_u32(smem + OFF_V + i * TILE_BYTES), HALF, 1024);
+      // K step k of a K-major 128-byte-swizzled tile: (k / 4) 64-column halves + (k % 4) 32-byte slices
+      auto koff = [](int k) -> uint64_t { return (uint64_t)(((k >> 2) * HALF + (k & 3) * 32) >> 4); };
+      // K step k of the MN-major V tile: 16 key rows of 128 bytes
+      auto voff = [](int k) -> uint64_t { return (uint64_t)((k * 16 * 128) >> 4); };
+      const uint32_t tm_s[2] = {tmem, tmem + 128};
+      const uint32_t tm_o[2] = {tmem + 256, tmem + 384};
+      // O_t += P_t V_i ; P_t read from TMEM columns [t*128, t*128 + 64)
+      auto issue_pv = [&](int t, int i) -> bool {
+        if (!mbar_wait(&p_full[t], i & 1, abort_flag, p.err)) return false;
+        if (t == 0 && !mbar_wait(&v_full[i & 1], (i >> 1) & 1, abort_flag, p.err)) return false;
+        tc_fence_after();
+        const uint64_t vb = dv[i & 1];
+        const uint32_t d = tm_o[t], pa = tm_s[t];
+        umma_bf16_ts(d, pa, vb, id_o, i != 0 ? 1u : 0u);
+  #pragma unroll
+        for (int k = 1; k < TILE / 16; ++k) umma_bf16_ts(d, pa + k * 8, vb + voff(k), id_o, 1u);
+        return true;
+      };
+      // S_t = Q_t K_j^T into TMEM columns [t*128, t*128 + 128)
+      auto issue_s = [&](int t, int j) {
+        const uint64_t kb = dk[j & 1], qb = dq[t];
+        const uint32_t d = tm_s[t];
+        umma_bf16_ss(d, qb, kb, id_s, 0u);
+  #pragma unroll
+        for (int k = 1; k < HD / 16; ++k) umma_bf16_ss(d, qb + koff(k), kb + koff(k), id_s, 1u);
+        umma_commit(&s_full[t]);
+      };
+      bool ok = mbar_wait(&q_full[0], 0, abort_flag, p.err);
+      for (int j = 0; ok && j < n_kv; ++j) {
+        if (!mbar_wait(&k_full[j & 1], (j >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
+        tc_fence_after();
+        if (j > 0 && !issue_pv(0, j - 1)) { ok = false; break; }
+        issue_s(0, j);
+        if (j > 0) {
+          if (!issue_pv(1, j - 1)) { ok = false; break; }
+          umma_commit(&v_empty[(j - 1) & 1]);
+        }
+        if (j == 0 && !mbar_wait(&q_full[1], 0, abort_flag, p.err)) { ok = false; break; }
+        issue_s(1, j);
+        umma_commit(&k_empty[j & 1]);
+      }
+      if (ok && issue_pv(0, n_kv - 1)) {
+        umma_commit(&o_full[0]);
+        if (issue_pv(1, n_kv - 1)) {
+          umma_commit(&o_full[1]);
+          umma_commit(&v_empty[(n_kv - 1) & 1]);
+        }
+      }
+      umma_commit(mma_done);
       int dummy = 0;
-      mbar_wait(&q_full[0], 0, &dummy);
-      if (nk_issued > 0) mbar_wait(&q_full[1], 0, &dummy);
-      for (int j = (nk_issued > 2 ? nk_issued - 2 : 0); j < nk_issued; ++j)
-        mbar_wait(&k_full[j & 1], (j >> 1) & 1, &dummy);
-      for (int j = (nv_issued > 2 ? nv_issued - 2 : 0); j < nv_issued; ++j)
-        mbar_wait(&v_full[j & 1], (j >> 1) & 1, &dummy);
+      mbar_wait(mma_done, 0, &dummy);
     }
-  } else if (warp == WARP_MMA && lane == 0) {
-    // ------------------------------------------------------------ MMA issuer
-    // Each UMMA here is only 64 tensor clocks of work, so the issuing thread must do
-    // almost nothing per instruction: every shared-memory descriptor is precomputed
-    // (a descriptor is linear in the address: desc(addr + off) = desc(addr) + off / 16).
-    const uint32_t id_s = idesc_bf16_f32(TILE, TILE);             // Q, K both K-major
-    const uint32_t id_o = idesc_bf16_f32(TILE, HD, false, true);  // P from TMEM, V MN-major
-    uint64_t dq[2], dk[2], dv[2];
-    for (int t = 0; t < 2; ++t) dq[t] = sdesc_kmajor_sw128(smem_u32(smem + OFF_Q + t * TILE_BYTES));
-    for (int i = 0; i < 2; ++i) dk[i] = sdesc_kmajor_sw128(smem_u32(smem + OFF_K + i * TILE_BYTES));
-    for (int i = 0; i < 2; ++i) dv[i] = sdesc_mnmajor_sw128(smem_u32(smem + OFF_V + i * TILE_BYTES), HALF, 1024);
-    // K step k of a K-major 128-byte-swizzled tile: (k / 4) 64-column halves + (k % 4) 32-byte slices
-    auto koff = [](int k) -> uint64_t { return (uint64_t)(((k >> 2) * HALF + (k & 3) * 32) >> 4); };
-    // K step k of the MN-major V tile: 16 key rows of 128 bytes
-    auto voff = [](int k) -> uint64_t { return (uint64_t)((k * 16 * 128) >> 4); };
-    const uint32_t tm_s[2] = {tmem, tmem + 128};
-    const uint32_t tm_o[2] = {tmem + 256, tmem + 384};
-    // O_t += P_t V_i ; P_t read from TMEM columns [t*128, t*128 + 64)
-    auto issue_pv = [&](int t, int i) -> bool {
-      if (!mbar_wait(&p_full[t], i & 1, abort_flag, p.err)) return false;
-      if (t == 0 && !mbar_wait(&v_full[i & 1], (i >> 1) & 1, abort_flag, p.err)) return false;
-      tc_fence_after();
-      const uint64_t vb = dv[i & 1];
-      const uint32_t d = tm_o[t], pa = tm_s[t];
-      umma_bf16_ts(d, pa, vb, id_o, i != 0 ? 1u : 0u);
-#pragma unroll
-      for (int k = 1; k < TILE / 16; ++k) umma_bf16_ts(d, pa + k * 8, vb + voff(k), id_o, 1u);
-      return true;
-    };
-    // S_t = Q_t K_j^T into TMEM columns [t*128, t*128 + 128)
-    auto issue_s = [&](int t, int j) {
-      const uint64_t kb = dk[j & 1], qb = dq[t];
-      const uint32_t d = tm_s[t];
-      umma_bf16_ss(d, qb, kb, id_s, 0u);
-#pragma unroll
-      for (int k = 1; k < HD / 16; ++k) umma_bf16_ss(d, qb + koff(k), kb + koff(k), id_s, 1u);
-      umma_commit(&s_full[t]);
-    };
-    bool ok = mbar_wait(&q_full[0], 0, abort_flag, p.err);
-    for (int j = 0; ok && j < n_kv; ++j) {
-      if (!mbar_wait(&k_full[j & 1], (j >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
-      tc_fence_after();
-      if (j > 0 && !issue_pv(0, j - 1)) { ok = false; break; }
-      issue_s(0, j);
-      if (j > 0) {
-        if (!issue_pv(1, j - 1)) { ok = false; break; }
-        umma_commit(&v_empty[(j - 1) & 1]);
-      }
-      if (j == 0 && !mbar_wait(&q_full[1], 0, abort_flag, p.err)) { ok = false; break; }
-      issue_s(1, j);
-      umma_commit(&k_empty[j & 1]);
-    }
-    if (ok && issue_pv(0, n_kv - 1)) {
-      umma_commit(&o_full[0]);
-      if (issue_pv(1, n_kv - 1)) {
-        umma_commit(&o_full[1]);
-        umma_commit(&v_empty[(n_kv - 1) & 1]);
-      }
-    }
-    umma_commit(mma_done);
-    int dummy = 0;
-    mbar_wait(mma_done, 0, &dummy);
-  } else if (warp < 8) {
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 208;\n" ::: "memory");
     // ------------------------------------------------------------ softmax
     const int t = warp >> 2;         // query tile of this warpgroup
     const int lg = warp & 3;         // TMEM lane group
