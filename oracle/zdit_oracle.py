@@ -40,11 +40,15 @@ Readings where the pages are silent (each is also listed in the design notes):
   R9  QK-norm (per-head RMSNorm of q and k before RoPE) is an option, off by default.
 
 Pins: every function is checked in tests/test_oracle.py against library routines, brute
-force, closed forms, invariants or values printed on the pages.  stack_forward and sample:
-parity unpinned as a whole (the pages print no output value); their parts are pinned, and so
-are stack-level invariants (zero projections reduce the stack to embed + final layer, branch
-isolation, captions acting only through the main blocks) and sampler invariants (schedule,
-telescoping Euler steps, negated CFG cases).
+force, closed forms, invariants or values printed on the pages.  stack_forward and sample
+(the pages print no output value for them) are checked against a composition of torch library
+routines (F.linear, F.rms_norm, F.layer_norm, scaled_dot_product_attention, complex-form RoPE,
+reshape/permute patchify) on tiny configurations; the block order, the packing and the
+positions are written there independently, so a reading of the pages shared by both sides is
+the one thing those tests cannot catch.  Stack-level invariants (zero projections reduce the
+stack to embed + final layer, branch isolation, captions acting only through the main blocks)
+and sampler invariants (schedule values, telescoping Euler steps, negated CFG cases) are pinned
+as well.
 """
 from __future__ import annotations
 

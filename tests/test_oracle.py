@@ -479,3 +479,111 @@ def test_captions_reach_the_image_only_through_main_blocks():
     other = dict(case, caps=case["caps"] + 0.5)
     np.testing.assert_allclose(O.stack_forward(other, Wm, d), O.stack_forward(case, Wm, d), rtol=0, atol=0)
     assert np.abs(O.stack_forward(other, W, d) - O.stack_forward(case, W, d)).max() > 1e-6
+
+
+# -------------------------------------------- stack and sampler against torch routines
+def _torch_temb(t, W, dim):
+    t64 = lambda a: torch.as_tensor(np.asarray(a, np.float64))
+    half = dim // 2
+    freqs = torch.exp(-math.log(10000.0) * torch.arange(half, dtype=torch.float64) / half)
+    args = 1000.0 * t64(t).reshape(-1)[:, None] * freqs[None, :]
+    emb = torch.cat([torch.cos(args), torch.sin(args)], dim=1)
+    return F.linear(F.silu(F.linear(emb, t64(W["w_t1"]), t64(W["b_t1"]))), t64(W["w_t2"]), t64(W["b_t2"]))
+
+
+def _torch_stack(d, W, case, flags=O.Flags()):
+    """The whole forward composed from torch library routines: F.linear embedders,
+    F.rms_norm caption norm, the blocks of _torch_block (rms_norm, complex-form RoPE,
+    scaled_dot_product_attention, silu), F.layer_norm final layer; positions, packing and
+    the block order are written here with torch indexing, not taken from the oracle."""
+    t64 = lambda a: torch.as_tensor(np.asarray(a, np.float64))
+    gh, gw = case["grid"]
+    n_img = gh * gw
+    n_caps, n_valids = list(case["n_caps"]), list(case["n_valids"])
+    B = len(n_caps)
+    temb = _torch_temb(case["t"], W, d.temb_dim)
+    x_img = [F.linear(t64(case["patches"][b]), t64(W["w_x"]), t64(W["b_x"])) for b in range(B)]
+    caps = t64(case["caps"])
+    x_cap, off = [], 0
+    for b in range(B):
+        c = torch.empty(n_caps[b], d.dim, dtype=torch.float64)
+        rows = caps[off:off + n_valids[b]]
+        c[:n_valids[b]] = F.linear(F.rms_norm(rows, (rows.shape[1],), weight=t64(W["w_capnorm"]), eps=1e-5),
+                                   t64(W["w_cap"]), t64(W["b_cap"]))
+        c[n_valids[b]:] = t64(W["pad_vec"])
+        x_cap.append(c)
+        off += n_valids[b]
+    hh, ww = torch.meshgrid(torch.arange(gh), torch.arange(gw), indexing="ij")
+    img_pos = [torch.stack([torch.full((n_img,), n_caps[b] + 1), hh.reshape(-1), ww.reshape(-1)], 1)
+               for b in range(B)]
+    cap_pos = [torch.stack([torch.arange(1, n_caps[b] + 1), torch.zeros(n_caps[b], dtype=torch.long),
+                            torch.zeros(n_caps[b], dtype=torch.long)], 1) for b in range(B)]
+    cum = lambda lens: np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+
+    def run(x, lens, pos, wb, fl):
+        blk = {"weights": wb, "x": x.numpy(), "cu_seqlens": cum(lens), "pos": pos.numpy(),
+               "temb": temb.numpy()}
+        return torch.from_numpy(_torch_block(d, blk, fl))
+
+    fl_ctx = O.Flags(adaln=False, sandwich=flags.sandwich, qk_norm=flags.qk_norm, tanh_gate=flags.tanh_gate)
+    xi, xc = torch.cat(x_img), torch.cat(x_cap)
+    for wb, kind in zip(W["blocks"], W["block_kinds"]):
+        if kind == "noise":
+            xi = run(xi, [n_img] * B, torch.cat(img_pos), wb, flags)
+        elif kind == "context":
+            xc = run(xc, n_caps, torch.cat(cap_pos), wb, fl_ctx)
+    cap_cu = cum(n_caps)
+    xj = torch.cat([torch.cat([xi[b * n_img:(b + 1) * n_img], xc[cap_cu[b]:cap_cu[b + 1]]]) for b in range(B)])
+    pj = torch.cat([torch.cat([img_pos[b], cap_pos[b]]) for b in range(B)])
+    lens = [n_img + c for c in n_caps]
+    for wb, kind in zip(W["blocks"], W["block_kinds"]):
+        if kind == "main":
+            xj = run(xj, lens, pj, wb, flags)
+    cu = cum(lens)
+    out = []
+    for b in range(B):
+        x = xj[cu[b]:cu[b] + n_img]
+        scale = F.linear(temb[b], t64(W["w_fada"]), t64(W["b_fada"]))
+        a = F.layer_norm(x, (x.shape[-1],), eps=1e-6) * (1.0 + scale)
+        out.append(F.linear(a, t64(W["w_final"]), t64(W["b_final"])))
+    return torch.stack(out).numpy()
+
+
+def test_stack_matches_torch_composition():
+    d, W, case = _tiny_stack(seed=11, n_noise=2, n_context=2, n_main=2)
+    np.testing.assert_allclose(O.stack_forward(case, W, d), _torch_stack(d, W, case), rtol=1e-9, atol=1e-9)
+
+
+def test_stack_matches_torch_composition_qk_norm_no_sandwich():
+    d = synth.BlockDims(dim=256, n_heads=2, head_dim=128, ffn_hidden=384)
+    W = synth.stack_weights(12, d, n_noise=1, n_context=1, n_main=2, cap_dim=64, qk_norm=True)
+    case = synth.stack_case(12, 4, 2, [32, 64], [1, 50], [0.9, 0.2], cap_dim=64)
+    fl = O.Flags(sandwich=False, qk_norm=True)
+    np.testing.assert_allclose(O.stack_forward(case, W, d, fl), _torch_stack(d, W, case, fl),
+                               rtol=1e-9, atol=1e-9)
+
+
+def test_sampler_matches_torch_composition():
+    # the 8-step loop composed with torch: closed-form schedule, patchify by reshape /
+    # permute, negated CFG and Euler with torch arithmetic, the forward of _torch_stack
+    d, W, _ = _tiny_stack(seed=13)
+    C, h, w = 16, 2, 3
+    latent = synth.latent_noise(13, (C, 2 * h, 2 * w))
+    caps_c = RNG.standard_normal((40, 64)).astype(np.float32)
+    caps_u = RNG.standard_normal((1, 64)).astype(np.float32)
+    cond = {"caps": caps_c, "n_cap": 64, "n_valid": 40}
+    unc = {"caps": caps_u, "n_cap": 32, "n_valid": 1}
+    g = 1.5
+    got = O.sample(latent, cond, unc, W, d, g=g, n_steps=8)
+    u = torch.arange(9, dtype=torch.float64) / 8
+    sig = 3 * (1 - u) / (3 * (1 - u) + u)
+    z = torch.as_tensor(latent, dtype=torch.float64).view(C, h, 2, w, 2).permute(1, 3, 2, 4, 0).reshape(h * w, 4 * C)
+    for i in range(8):
+        case = {"grid": (h, w), "patches": torch.stack([z, z]).numpy(),
+                "caps": np.concatenate([caps_c, caps_u]), "n_caps": [64, 32], "n_valids": [40, 1],
+                "t": np.array([1 - sig[i].item()] * 2)}
+        out = torch.from_numpy(_torch_stack(d, W, case))
+        v = -(out[0] + g * (out[0] - out[1]))
+        z = z + (sig[i + 1] - sig[i]) * v
+    ref = z.reshape(h, w, 2, 2, C).permute(4, 0, 2, 1, 3).reshape(C, 2 * h, 2 * w).numpy()
+    np.testing.assert_allclose(got, ref, rtol=1e-9, atol=1e-9)
