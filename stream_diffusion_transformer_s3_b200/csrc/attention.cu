@@ -269,7 +269,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ------------------------------------------------------------ softmax
     const int t = warp >> 2;         // query tile of this warpgroup
     const int lg = warp & 3;         // TMEM lane group
-    const int row = lg * 32 + lane;  // query row inside the tile == TMEM lane
     const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
     const uint32_t tS = tmem + lane_off + t * 128;
     const uint32_t tO = tmem + lane_off + 256 + t * 128;
