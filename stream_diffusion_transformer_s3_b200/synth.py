@@ -58,10 +58,15 @@ def randn(seed: int, tensor_id: int, shape, std: float = 1.0) -> np.ndarray:
 
 
 def bf16_round(x: np.ndarray) -> np.ndarray:
-    """float32 -> nearest bfloat16 value (ties to even), returned as float32."""
-    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
-    u = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
-    return u.astype(np.uint32).view(np.float32)
+    """float32 -> nearest bfloat16 value (ties to even), returned as float32.
+    (uint32 arithmetic wraps like the truncation of a wider sum, so every input maps to
+    the same bits as adding in 64 bits and keeping the low 32.)"""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    r = (u >> np.uint32(16)) & np.uint32(1)
+    r += np.uint32(0x7FFF)
+    r += u
+    r &= np.uint32(0xFFFF0000)
+    return r.view(np.float32)
 
 
 def bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -90,22 +95,30 @@ def block_weights(seed: int, block_index: int, d: BlockDims, adaln: bool = True,
     w_qkv [3D, D] (rows q | k | v, head h at rows h*128 .. h*128+127 of each),
     w_out [D, D], w1 (gate) [F, D], w3 (up) [F, D], w2 [D, F], w_ada [4D, E], b_ada [4D].
     """
-    D, F, E, dh = d.dim, d.ffn_hidden, d.temb_dim, d.head_dim
-    t = lambda name: block_index * 64 + _BLOCK_TID[name]
-    g = lambda name, shape: bf16_round(randn(seed, t(name), shape, 0.02))
-    w = {
-        "w_qkv": g("w_qkv", (3 * D, D)), "w_out": g("w_out", (D, D)),
-        "w1": g("w1", (F, D)), "w3": g("w3", (F, D)), "w2": g("w2", (D, F)),
-    }
-    for n in ("n_attn", "n_attn_post", "n_ffn", "n_ffn_post"):
-        w[n] = (1.0 + randn(seed, t(n), (D,), 0.1)).astype(np.float32)
+    names = ["w_qkv", "w_out", "w1", "w3", "w2", "n_attn", "n_attn_post", "n_ffn", "n_ffn_post"]
     if qk_norm:
-        w["n_q"] = (1.0 + randn(seed, t("n_q"), (dh,), 0.1)).astype(np.float32)
-        w["n_k"] = (1.0 + randn(seed, t("n_k"), (dh,), 0.1)).astype(np.float32)
+        names += ["n_q", "n_k"]
     if adaln:
-        w["w_ada"] = g("w_ada", (4 * D, E))
-        w["b_ada"] = randn(seed, t("b_ada"), (4 * D,), 0.02)
-    return w
+        names += ["w_ada", "b_ada"]
+    return {n: block_tensor(seed, block_index, d, n) for n in names}
+
+
+def block_tensor(seed: int, block_index: int, d: BlockDims, name: str) -> np.ndarray:
+    """One tensor of block_weights(seed, block_index, d, ...), drawn on its own (each
+    tensor has its own stream, so drawing one alone gives the same values)."""
+    D, F, E, dh = d.dim, d.ffn_hidden, d.temb_dim, d.head_dim
+    tid = block_index * 64 + _BLOCK_TID[name]
+    gemm_shapes = {"w_qkv": (3 * D, D), "w_out": (D, D), "w1": (F, D), "w3": (F, D), "w2": (D, F),
+                   "w_ada": (4 * D, E)}
+    if name in gemm_shapes:
+        return bf16_round(randn(seed, tid, gemm_shapes[name], 0.02))
+    if name in ("n_attn", "n_attn_post", "n_ffn", "n_ffn_post"):
+        return (1.0 + randn(seed, tid, (D,), 0.1)).astype(np.float32)
+    if name in ("n_q", "n_k"):
+        return (1.0 + randn(seed, tid, (dh,), 0.1)).astype(np.float32)
+    if name == "b_ada":
+        return randn(seed, tid, (4 * D,), 0.02)
+    raise KeyError(name)
 
 
 def stack_weights(seed: int, d: BlockDims, n_noise: int = 2, n_context: int = 2,
