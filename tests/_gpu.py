@@ -1,9 +1,12 @@
 """Shared helpers of the GPU parity tests (device marshalling and error metrics)."""
+from collections.abc import Mapping
+
 import numpy as np
 import pytest
 import torch
 
 import stream_diffusion_transformer_s3_b200 as Z
+from stream_diffusion_transformer_s3_b200 import synth
 
 
 def require_gpu():
@@ -62,3 +65,55 @@ def run_block_gpu(case, d, flags):
     Z.zdit_block_forward(dims, fl, w, vl, x, temb, cs, sn, ws)
     assert Z.zdit_device_status() == 0
     return host(x)
+
+
+def run_stack(W, case, d, n_noise, n_ctx, n_main, cap_dim, flags=Z.F_ADALN | Z.F_SANDWICH_NORM, blocks=None):
+    dims = dims_of(d)
+    st = Z.DeviceStack(W, dims, n_noise, n_ctx, n_main, patch_dim=64, cap_dim=cap_dim, flags=flags, blocks=blocks)
+    call = Z.StackCall(case["grid"], case["n_caps"], case["n_valids"], case["t"], dev(case["patches"]),
+                       dev(case["caps"]))
+    ws = torch.empty(Z.stack_workspace_bytes(st, call), dtype=torch.uint8, device="cuda")
+    out = torch.full((len(case["n_caps"]), case["grid"][0] * case["grid"][1], 64), float("nan"), device="cuda")
+    Z.zdit_stack_forward(st, call, out, ws)
+    assert Z.zdit_device_status() == 0
+    return host(out)
+
+
+class BlockSource:
+    """Draws each block's weights once: the first read of block i draws all its tensors,
+    uploads them for the GPU and keeps the host copy only until another block is read, so
+    the 34 full-width blocks (12 GB as bf16) never sit on the host at once."""
+
+    def __init__(self, seed, d, kinds):
+        self.seed, self.d, self.kinds = seed, d, kinds
+        self.device = [None] * len(kinds)
+        self.current = (None, None)
+
+    def host(self, i):
+        if self.current[0] != i:
+            w = synth.block_weights(self.seed, i, self.d, adaln=self.kinds[i] != "context")
+            if self.device[i] is None:
+                self.device[i] = Z.DeviceBlock(w)
+            self.current = (i, w)
+        return self.current[1]
+
+
+class LazyBlock(Mapping):
+    """Block i's weights as the oracle reads them, drawn by a BlockSource on first use."""
+
+    def __init__(self, source, i):
+        self.source, self.i = source, i
+        self.names = ["w_qkv", "w_out", "w1", "w3", "w2", "n_attn", "n_attn_post", "n_ffn", "n_ffn_post"]
+        if source.kinds[i] != "context":
+            self.names += ["w_ada", "b_ada"]
+
+    def __getitem__(self, name):
+        if name not in self.names:
+            raise KeyError(name)
+        return self.source.host(self.i)[name]
+
+    def __iter__(self):
+        return iter(self.names)
+
+    def __len__(self):
+        return len(self.names)

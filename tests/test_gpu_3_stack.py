@@ -1,15 +1,10 @@
 """Stack-level parity on the GPU: zdit_stack_forward (embedders, noise and context
 refiners, joint main blocks, final layer) against the oracle's stack_forward."""
-from collections.abc import Mapping
-
-import numpy as np
 import pytest
-import torch
 
 import oracle as O
-import stream_diffusion_transformer_s3_b200 as Z
 from stream_diffusion_transformer_s3_b200 import synth
-from _gpu import dev, dims_of, errors, host, require_gpu
+from _gpu import BlockSource, LazyBlock, errors, require_gpu, run_stack
 
 pytestmark = pytest.mark.gpu
 
@@ -17,18 +12,6 @@ pytestmark = pytest.mark.gpu
 @pytest.fixture(autouse=True)
 def _gpu():
     require_gpu()
-
-
-def run_stack(W, case, d, n_noise, n_ctx, n_main, cap_dim, flags=Z.F_ADALN | Z.F_SANDWICH_NORM, blocks=None):
-    dims = dims_of(d)
-    st = Z.DeviceStack(W, dims, n_noise, n_ctx, n_main, patch_dim=64, cap_dim=cap_dim, flags=flags, blocks=blocks)
-    call = Z.StackCall(case["grid"], case["n_caps"], case["n_valids"], case["t"], dev(case["patches"]),
-                       dev(case["caps"]))
-    ws = torch.empty(Z.stack_workspace_bytes(st, call), dtype=torch.uint8, device="cuda")
-    out = torch.full((len(case["n_caps"]), case["grid"][0] * case["grid"][1], 64), float("nan"), device="cuda")
-    Z.zdit_stack_forward(st, call, out, ws)
-    assert Z.zdit_device_status() == 0
-    return host(out)
 
 
 @pytest.mark.parametrize("n_caps,n_valids", [((64, 32), (45, 1)), ((32,), (0,))])
@@ -55,46 +38,6 @@ def test_full_width_stack_two_blocks_per_kind_256px():
     assert e["rel_l2"] <= 2e-2, e
 
 
-class _BlockSource:
-    """Draws each block's weights once: the first read of block i draws all its tensors,
-    uploads them for the GPU and keeps the host copy only until another block is read, so
-    the 34 full-width blocks (12 GB as bf16) never sit on the host at once."""
-
-    def __init__(self, seed, d, kinds):
-        self.seed, self.d, self.kinds = seed, d, kinds
-        self.device = [None] * len(kinds)
-        self.current = (None, None)
-
-    def host(self, i):
-        if self.current[0] != i:
-            w = synth.block_weights(self.seed, i, self.d, adaln=self.kinds[i] != "context")
-            if self.device[i] is None:
-                self.device[i] = Z.DeviceBlock(w)
-            self.current = (i, w)
-        return self.current[1]
-
-
-class _LazyBlock(Mapping):
-    """Block i's weights as the oracle reads them, drawn by a _BlockSource on first use."""
-
-    def __init__(self, source, i):
-        self.source, self.i = source, i
-        self.names = ["w_qkv", "w_out", "w1", "w3", "w2", "n_attn", "n_attn_post", "n_ffn", "n_ffn_post"]
-        if source.kinds[i] != "context":
-            self.names += ["w_ada", "b_ada"]
-
-    def __getitem__(self, name):
-        if name not in self.names:
-            raise KeyError(name)
-        return self.source.host(self.i)[name]
-
-    def __iter__(self):
-        return iter(self.names)
-
-    def __len__(self):
-        return len(self.names)
-
-
 def test_full_width_full_depth_stack_256px():
     # the whole 34-block stack (2 noise refiners, 2 context refiners, 30 main blocks) at
     # full width, free-running from the embedders to the final layer, 16x16 image grid,
@@ -104,9 +47,9 @@ def test_full_width_full_depth_stack_256px():
     seed = 21
     kinds = ["noise"] * 2 + ["context"] * 2 + ["main"] * 30
     W = synth.stack_weights(seed, d, blocks=False)
-    src = _BlockSource(seed, d, kinds)
+    src = BlockSource(seed, d, kinds)
     case = synth.stack_case(seed, 16, 16, [64, 32], [45, 1], [0.6, 0.6])
-    ref = O.stack_forward(case, dict(W, blocks=[_LazyBlock(src, i) for i in range(len(kinds))], block_kinds=kinds), d)
+    ref = O.stack_forward(case, dict(W, blocks=[LazyBlock(src, i) for i in range(len(kinds))], block_kinds=kinds), d)
     assert all(b is not None for b in src.device)
     got = run_stack(W, case, d, 2, 2, 30, 2560, blocks=src.device)
     e = errors(got, ref)

@@ -2,7 +2,11 @@
 bench.py times: one main block over the joint cond/uncond sequence (4224 + 4128
 tokens, width 3840) checked on sampled rows against the oracle; the attention-only
 sweep sizes checked on sampled query rows; the whole 34-block stack checked through
-properties that hold at any size (branch isolation, determinism, finiteness)."""
+properties that hold at any size (branch isolation, determinism, finiteness) and, on request
+(ZDIT_FULL_STACK_PARITY=1: the float64 oracle of the whole forward takes minutes of host
+time), free-running against the oracle."""
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -10,7 +14,7 @@ import torch
 import oracle as O
 import stream_diffusion_transformer_s3_b200 as Z
 from stream_diffusion_transformer_s3_b200 import synth
-from _gpu import bf16, dev, dims_of, errors, host, require_gpu, run_block_gpu
+from _gpu import BlockSource, LazyBlock, bf16, dev, dims_of, errors, host, require_gpu, run_block_gpu, run_stack
 
 pytestmark = pytest.mark.gpu
 TOL = 2e-2
@@ -124,3 +128,22 @@ def test_fullsize_stack_branch_isolation_and_determinism():
     assert torch.equal(both[1], unc[0])
     # the two branches differ (different captions)
     assert (both[0] - both[1]).abs().max().item() > 1e-3
+
+
+@pytest.mark.skipif(os.environ.get("ZDIT_FULL_STACK_PARITY") != "1",
+                    reason="the float64 oracle of the whole 1024x1024 forward takes ~7 min of host time")
+def test_fullsize_stack_free_running():
+    # the benchmarked workload end to end: 64x64 image grid per branch, captions 128 (100 valid)
+    # and 32 (1 valid), 2 + 2 + 30 full-width blocks, embedders and final layer, against the
+    # oracle's stack_forward on the same inputs
+    d = synth.FULL
+    seed = 31
+    kinds = ["noise"] * 2 + ["context"] * 2 + ["main"] * 30
+    W = synth.stack_weights(seed, d, blocks=False)
+    src = BlockSource(seed, d, kinds)
+    case = synth.stack_case(seed, 64, 64, [128, 32], [100, 1], [0.5, 0.5])
+    ref = O.stack_forward(case, dict(W, blocks=[LazyBlock(src, i) for i in range(len(kinds))], block_kinds=kinds), d)
+    got = run_stack(W, case, d, 2, 2, 30, 2560, blocks=src.device)
+    e = errors(got, ref)
+    print("\nstack 1024x1024, 34 blocks, free-running", e)
+    assert e["rel_l2"] <= TOL, e
