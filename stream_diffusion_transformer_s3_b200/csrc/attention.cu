@@ -22,8 +22,9 @@
 // PV_t(j-1) is issued before S_t(j), the commit that signals S_t(j) also proves that
 // PV_t(j-1) is done: the softmax may then overwrite P_t and rescale O_t freely.
 // Online softmax in FP32 with a lazily moved reference max: the running max only
-// moves (and O is rescaled) when a row's max grows by more than 2^8, so the common
-// tile needs no O round trip; P = exp2(s - m_ref) <= 256 stays in bf16 range.
+// moves (and O is rescaled) when a row's max grows by more than 16 (log2 units), so
+// the common tile needs no O round trip; P = exp2(s - m_ref) <= 2^16 keeps bf16's
+// relative precision, and O and the row sum stay far inside FP32 range.
 // The epilogue stages O / l as bf16 in the shared memory that Q and the K ring no
 // longer need, then writes two full 256-byte rows per warp store instruction.
 #include <cstdio>
@@ -50,7 +51,7 @@ constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
 constexpr int OFF_V = OFF_K + 2 * TILE_BYTES;
 constexpr int OFF_BAR = OFF_V + 2 * TILE_BYTES;
 constexpr int SMEM_BYTES = 1024 + OFF_BAR + 256;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr float kRescaleThreshold = 16.0f;  // log2 units
 
 struct AParams {
   int ldo, n_heads, batch;
