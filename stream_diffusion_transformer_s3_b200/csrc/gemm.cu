@@ -13,8 +13,9 @@
 // Epilogues (the DiT block's projection steps, "Z-Image-Turbo port" DiT row and
 // "Native creative jobs", "Recipes and precision": FP32 accumulators, SwiGLU gate in
 // FP32, bf16 storage, never fp16):
-//   EPI_F32    fp32 store (+ bias)                 out-proj, w2, embedders
-//   EPI_BF16   bf16 store (+ bias)
+//   EPI_F32    fp32 store (+ bias)                 embedders, final layer
+//   EPI_BF16   bf16 store (+ bias)                 out-proj, w2 (y, normalized in FP32
+//                                                  by the residual kernel)
 //   EPI_QKV    q/k columns: real interleaved RoPE with per-token cos/sin, 32-column
 //              chunks; bf16 store of [q | k | v]
 //   EPI_QKV_NORM  same with a per-head RMSNorm of q and k first (whole head at once)
