@@ -56,7 +56,7 @@ def forward_flops() -> float:
 # DRAM bytes per launch of the dominant kernel (gate/up GEMM of a main block, 8352 x 20480
 # x 3840), from one ncu capture (profiles/gemm_gate_up_swiglu_block_1024.md), valid for the
 # GEMM sources with this hash only; any change to them makes the figure stale (reported null).
-NCU_TRAFFIC = {"kernel": "gemm_gate_up_swiglu", "bytes": 417948928 + 155953152, "src_hash": "7b9819d2321a963c"}
+NCU_TRAFFIC = {"kernel": "gemm_gate_up_swiglu", "bytes": 415824896 + 156079616, "src_hash": "f26bc7eb487c1460"}
 
 
 def gemm_src_hash() -> str:

@@ -377,23 +377,37 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 // ------------------------------------------------------------------------------
 // CTA-pair variant (cta_group::2): a cluster of two CTAs computes a 256 x 256 tile.
-// Each CTA TMA-loads its own 128 rows of A and its own 128 rows of B per 64-deep
-// k-slice (32 KB per stage, 6 stages) and counts the bytes on the leader's barrier;
+// Each CTA TMA-loads its own 128 rows of A and its own 128 rows of B per k-slice and
+// counts the bytes on the leader's barrier;
 // the leader's single MMA thread issues M=256 x N=256 MMAs that read both CTAs'
 // shared memory and write 128 rows x 256 columns into each CTA's TMEM; commits are
 // multicast to both CTAs.  Each CTA runs the same epilogue on its 128 rows.  Per
-// SM this halves the B traffic and gives the ring 50% more stages than the single
-// CTA kernel.  No TMA multicast is used.
-constexpr int P_STAGES = 6;
-constexpr int P_A_TILE = 128 * BK * 2;  // 16 KB
-constexpr int P_B_TILE = 128 * BK * 2;  // 16 KB
-constexpr int P_STAGE_BYTES = P_A_TILE + P_B_TILE;
-constexpr int P_SMEM_BYTES = 1024 + P_STAGES * P_STAGE_BYTES + 256;
+// SM this halves the B traffic.  No TMA multicast is used.
+// Ring: 192 KB either as 6 stages of 64-deep slices (32 KB) or as 3 stages of 128-deep
+// slices (two 64-column swizzled halves per operand, 64 KB), which give the MMA thread 8
+// UMMAs (1024 tensor clocks) per barrier wait instead of 4.  Measured per projection
+// (ncu, one main block): the gate/up GEMM runs its tensor pipe 94% of the time with
+// 128-deep slices against 89% with 64-deep ones; QKV and the out-projection (K = 3840)
+// lose 3-4 points with them; so the SwiGLU projection takes 128 and the others 64.
+template <int PBK>
+struct PairRing {
+  static constexpr int BKP = PBK;
+  static constexpr int STAGES = PBK == 128 ? 3 : 6;
+  static constexpr int A_TILE = 128 * PBK * 2;
+  static constexpr int B_TILE = 128 * PBK * 2;
+  static constexpr int STAGE_BYTES = A_TILE + B_TILE;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+};
+template <int EPI>
+__host__ __device__ constexpr int pair_bk() { return EPI == EPI_SWIGLU ? 128 : 64; }
 
 template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const KParams p) {
+  using Ring = PairRing<pair_bk<EPI>()>;
+  constexpr int P_BK = Ring::BKP, P_STAGES = Ring::STAGES, P_A_TILE = Ring::A_TILE;
+  constexpr int P_STAGE_BYTES = Ring::STAGE_BYTES;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + P_STAGES * P_STAGE_BYTES);
@@ -452,8 +466,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         uint8_t* sa = smem + stage * P_STAGE_BYTES;
         if (leader) mbar_arrive_expect_tx(&full[stage], 2 * P_STAGE_BYTES);
         const uint32_t bar = leader_smem_addr(&full[stage]);
-        tma_load_2d_pair(sa, &tmA, bar, kb * BK, m0);
-        tma_load_2d_pair(sa + P_A_TILE, &tmB, bar, kb * BK, n0);
+#pragma unroll
+        for (int h = 0; h < P_BK / 64; ++h) {
+          tma_load_2d_pair(sa + h * 16384, &tmA, bar, kb * P_BK + h * 64, m0);
+          tma_load_2d_pair(sa + P_A_TILE + h * 16384, &tmB, bar, kb * P_BK + h * 64, n0);
+        }
         armed |= 1u << stage;
         armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
         if (++stage == P_STAGES) {
@@ -489,9 +506,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const uint32_t a0 = smem_u32(smem + stage * P_STAGE_BYTES);
         const uint32_t b0 = a0 + P_A_TILE;
 #pragma unroll
-        for (int k = 0; k < BK / 16; ++k)
-          umma_pair_bf16_ss(d, sdesc_kmajor_sw128(a0 + k * 32), sdesc_kmajor_sw128(b0 + k * 32), idesc,
+        for (int k = 0; k < P_BK / 16; ++k) {
+          // K step k: (k / 4) 64-column swizzled halves of 16 KB + (k % 4) 32-byte slices
+          const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+          umma_pair_bf16_ss(d, sdesc_kmajor_sw128(a0 + off), sdesc_kmajor_sw128(b0 + off), idesc,
                             (kb | k) != 0 ? 1u : 0u);
+        }
         umma_pair_commit_mc(&empty[stage], 0x3);
         if (++stage == P_STAGES) {
           stage = 0;
@@ -558,12 +578,14 @@ zdit_status launch_epi(const CUtensorMap& ta, const CUtensorMap& tb, const KPara
   static bool attr_set = false, attr_pair_set = false;
   if (pair) {
     if (!attr_pair_set) {
-      if (cudaFuncSetAttribute(gemm_pair_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_BYTES) !=
+      if (cudaFuncSetAttribute(gemm_pair_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               PairRing<pair_bk<EPI>()>::SMEM_BYTES) !=
           cudaSuccess)
         return ZDIT_ERR_CUDA;
       attr_pair_set = true;
     }
-    launch_dependent(gemm_pair_kernel<EPI>, dim3(grid), dim3(THREADS), P_SMEM_BYTES, s, ta, tb, kp);
+    launch_dependent(gemm_pair_kernel<EPI>, dim3(grid), dim3(THREADS), PairRing<pair_bk<EPI>()>::SMEM_BYTES, s, ta, tb,
+                     kp);
   } else {
     if (!attr_set) {
       if (cudaFuncSetAttribute(gemm_tc_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
@@ -624,7 +646,8 @@ zdit_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
   kp.rcos = a.rope_cos; kp.rsin = a.rope_sin; kp.qn = a.qn; kp.kn = a.kn; kp.eps = a.eps; kp.dim = a.dim;
   kp.num_m = pair ? (a.M + 255) / 256 : (a.M + BM - 1) / BM;
   kp.num_n = (a.N + BN - 1) / BN;
-  kp.num_k = (a.K + BK - 1) / BK;
+  const int kslice = !pair ? BK : (a.epi == EPI_SWIGLU ? pair_bk<EPI_SWIGLU>() : pair_bk<EPI_BF16>());
+  kp.num_k = (a.K + kslice - 1) / kslice;
   // L2-aware raster: a band of tiles of one operand (about 32 MB, well inside one
   // die's share of the L2) stays resident while the other operand streams; the
   // streamed operand is re-read once per band.
