@@ -100,6 +100,7 @@ struct BlockWs {
   __nv_bfloat16* qkvh;  // [T, max(3D, F)]
   __nv_bfloat16* o;     // [T, D]
   __nv_bfloat16* y;     // [T, D] projection output before the sandwich norm
+  int* bands;           // [2 ceil(T / 256)] arrival counters of the out / down projections
 };
 
 size_t carve_block(Carver& c, BlockWs* ws, int64_t T, int B, int D, int F) {
@@ -110,6 +111,7 @@ size_t carve_block(Carver& c, BlockWs* ws, int64_t T, int B, int D, int F) {
   w.qkvh = c.take<__nv_bfloat16>((size_t)T * wide);
   w.o = c.take<__nv_bfloat16>((size_t)T * D);
   w.y = c.take<__nv_bfloat16>((size_t)T * D);
+  w.bands = c.take<int>((size_t)(T + 255) / 256 * 2);  // one per 128-row half of every 256-row pair tile
   if (ws) *ws = w;
   return c.off;
 }
@@ -125,6 +127,14 @@ bool varlen_ok(const zdit_varlen* v) {
 
 inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
+// Band counters of one forward: zeroed when the token count changes, then every
+// projection that signals them adds num_n arrivals per band, so the k-th one of the
+// run is complete for a band at k * num_n.
+struct BandState {
+  int T = -1;
+  int epoch = 0;
+};
+
 // Next block's pre-attention norm, fused into this block's last residual kernel.
 struct NextNorm {
   const float* w;      // next block's n_attn
@@ -137,7 +147,7 @@ struct NextNorm {
 // pre-attention norm into the final residual kernel.
 zdit_status run_block(const zdit_block_cfg& cfg, const zdit_block_weights& w, const zdit_varlen& vl, int T,
                       float* x, const float* mod, const float* rcos, const float* rsin, const BlockWs& ws,
-                      cudaStream_t s, bool a_ready = false, const NextNorm* next = nullptr) {
+                      cudaStream_t s, BandState* band, bool a_ready = false, const NextNorm* next = nullptr) {
   const int D = cfg.dim, F = cfg.ffn_hidden, B = vl.batch;
   const bool adaln = cfg.flags & ZDIT_F_ADALN;
   const bool sandwich = cfg.flags & ZDIT_F_SANDWICH_NORM;
@@ -147,6 +157,18 @@ zdit_status run_block(const zdit_block_cfg& cfg, const zdit_block_weights& w, co
   const float* s2 = adaln ? mod + 2 * D : nullptr;
   const float* g2 = adaln ? mod + 3 * D : nullptr;
   const int ms = 4 * D;
+  // The residual kernels start band by band while their projection finishes (needs the
+  // pair GEMM, and programmatic launches so the residual grid is resident early; off
+  // under the event profiler, which times kernels one by one).
+  const bool banded = band != nullptr && ws.bands != nullptr && gemm_uses_pair(T, D) && !profiling_on() &&
+                      pdl_enabled();
+  const int band_step = D / 256;  // arrivals per band per projection (N = D output tiles)
+  if (banded && band->T != T) {
+    if (cudaMemsetAsync(ws.bands, 0, (size_t)(T + 255) / 256 * 2 * sizeof(int), s) != cudaSuccess)
+      return ZDIT_ERR_CUDA;
+    band->T = T;
+    band->epoch = 0;
+  }
 
   // pre-attention norm + modulation -> bf16 operand
   if (!a_ready)
@@ -173,6 +195,7 @@ zdit_status run_block(const zdit_block_cfg& cfg, const zdit_block_weights& w, co
   GemmArgs go{};
   go.A = ws.o; go.lda = D; go.B = w.w_out; go.ldb = D; go.M = T; go.N = D; go.K = D;
   go.epi = EPI_BF16; go.out = ws.y; go.ldo = D; go.prof_kind = PROF_GEMM_OUT;
+  go.band_flags = banded ? ws.bands : nullptr;
   st = launch_gemm(go, s);
   if (st != ZDIT_OK) return st;
 
@@ -182,6 +205,8 @@ zdit_status run_block(const zdit_block_cfg& cfg, const zdit_block_weights& w, co
   r.gate = g1; r.gate_stride = ms; r.tanh_gate = (cfg.flags & ZDIT_F_TANH_GATE) ? 1 : 0;
   r.cu_seqlens = vl.cu_seqlens_dev; r.batch = B; r.eps = cfg.norm_eps;
   r.next_w = w.n_ffn; r.next_scale = s2; r.next_scale_stride = ms; r.next_out = ws.a;
+  r.band_flags = banded ? ws.bands : nullptr;
+  r.band_target = banded ? ++band->epoch * band_step : 0;
   launch_residual(r, s);
 
   // gate/up projection with SwiGLU epilogue -> h bf16 [T, F]
@@ -195,6 +220,7 @@ zdit_status run_block(const zdit_block_cfg& cfg, const zdit_block_weights& w, co
   GemmArgs gd{};
   gd.A = ws.qkvh; gd.lda = F; gd.B = w.w_down; gd.ldb = F; gd.M = T; gd.N = D; gd.K = F;
   gd.epi = EPI_BF16; gd.out = ws.y; gd.ldo = D; gd.prof_kind = PROF_GEMM_DOWN;
+  gd.band_flags = banded ? ws.bands : nullptr;
   st = launch_gemm(gd, s);
   if (st != ZDIT_OK) return st;
 
@@ -202,6 +228,7 @@ zdit_status run_block(const zdit_block_cfg& cfg, const zdit_block_weights& w, co
   ResidArgs r2 = r;
   r2.post_w = sandwich ? w.n_ffn_post : nullptr;
   r2.gate = g2;
+  r2.band_target = banded ? ++band->epoch * band_step : 0;
   if (next != nullptr) {
     r2.next_w = next->w; r2.next_scale = next->scale; r2.next_out = ws.a;
   } else {
@@ -386,6 +413,7 @@ zdit_status stack_run(const zdit_stack_cfg* cfg, const zdit_stack_weights* w, co
   }
 
   // refiners
+  BandState band;
   zdit_varlen v_img{B_img, ws.cu_img, d.cu_img};
   zdit_varlen v_cap{B, ws.cu_cap, d.cu_cap};
   zdit_varlen v_joint{B, ws.cu_joint, d.cu_joint};
@@ -397,8 +425,9 @@ zdit_status stack_run(const zdit_stack_cfg* cfg, const zdit_stack_weights* w, co
     zdit_block_cfg bc = bcfg;
     if (ctx) bc.flags &= ~ZDIT_F_ADALN;
     const float* mod = ws.mods + (size_t)i * B * 4 * D;
-    st = noise ? run_block(bc, w->blocks[i], v_img, B_img * d.n_img, ws.x_img, mod, ws.cos_img, ws.sin_img, ws.blk, s)
-               : run_block(bc, w->blocks[i], v_cap, d.T_cap, ws.x_cap, mod, ws.cos_cap, ws.sin_cap, ws.blk, s);
+    st = noise ? run_block(bc, w->blocks[i], v_img, B_img * d.n_img, ws.x_img, mod, ws.cos_img, ws.sin_img, ws.blk, s,
+                           &band)
+               : run_block(bc, w->blocks[i], v_cap, d.T_cap, ws.x_cap, mod, ws.cos_cap, ws.sin_cap, ws.blk, s, &band);
     if (st != ZDIT_OK) return st;
   }
   // concatenate each branch as [image | caption]
@@ -422,7 +451,7 @@ zdit_status stack_run(const zdit_stack_cfg* cfg, const zdit_stack_weights* w, co
       nn.scale = adaln ? ws.mods + (size_t)(i + 1) * B * 4 * D : nullptr;
     }
     st = run_block(bcfg, w->blocks[i], v_joint, d.T, ws.x_joint, ws.mods + (size_t)i * B * 4 * D, ws.cos_joint,
-                   ws.sin_joint, ws.blk, s, i > first_main, has_next ? &nn : nullptr);
+                   ws.sin_joint, ws.blk, s, &band, i > first_main, has_next ? &nn : nullptr);
     if (st != ZDIT_OK) return st;
   }
   // final layer on the image rows of each branch
@@ -488,7 +517,8 @@ ZDIT_API zdit_status zdit_block_forward(const zdit_block_cfg* cfg, const zdit_bl
   if (cfg->flags & ZDIT_F_ADALN)
     launch_gemv(static_cast<const __nv_bfloat16*>(w->w_ada), w->b_ada, temb, varlen->batch, cfg->temb_dim,
                 4 * cfg->dim, ws.mod, s);
-  return run_block(*cfg, *w, *varlen, T, x, ws.mod, rope_cos, rope_sin, ws, s);
+  BandState band;
+  return run_block(*cfg, *w, *varlen, T, x, ws.mod, rope_cos, rope_sin, ws, s, &band);
 }
 
 ZDIT_API size_t zdit_stack_workspace_bytes(const zdit_stack_cfg* cfg, const zdit_stack_inputs* in) {

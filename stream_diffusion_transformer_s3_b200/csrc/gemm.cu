@@ -57,6 +57,7 @@ struct KParams {
   int dim;
   int num_m, num_n, num_k, group_m, group_n, raster;
   int* err;
+  int* band_flags;  // per 128-row band arrival counters or nullptr
 };
 
 // Tile order of the persistent loop.  raster 0: bands of group_m M-tiles, M fastest
@@ -539,6 +540,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       tile_coords(t, p, mb, nb);
       const uint32_t taddr = tmem_base + ((uint32_t)(lg * 32) << 16) + acc * BN;
       epilogue_tile<EPI>(p, taddr, mb * 256 + (int)rank * 128 + lg * 32 + lane, nb);
+      if (p.band_flags != nullptr) {
+        // this CTA's 128 rows of the tile are stored: one arrival on their band
+        __threadfence();
+        named_bar_sync(1, 128);
+        if (warp == 2 && lane == 0) atomicAdd(p.band_flags + mb * 2 + (int)rank, 1);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -625,6 +632,8 @@ bool force_single_cta() {
   return v == 1;
 }
 
+bool gemm_uses_pair(int M, int N) { return M > 256 && N % BN == 0 && !force_single_cta(); }
+
 zdit_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
   if (a.M <= 0 || a.N <= 0 || a.K <= 0) return ZDIT_ERR_SHAPE;
   if (a.K % 8 || a.lda % 8 || a.ldb % 8 || a.N % 32) return ZDIT_ERR_SHAPE;
@@ -665,6 +674,7 @@ zdit_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
     kp.raster = traffic_m <= traffic_n ? 0 : 1;
   }
   kp.err = device_error_ptr();
+  kp.band_flags = pair ? a.band_flags : nullptr;
   const int tiles = kp.num_m * kp.num_n;
   int grid = tiles < num_sms() ? tiles : num_sms();
   if (pair) {

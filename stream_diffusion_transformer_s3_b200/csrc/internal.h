@@ -59,9 +59,15 @@ struct GemmArgs {
   const float* kn;
   float eps;
   int prof_kind = PROF_GEMM_OTHER;
+  // Optional per-128-row-band arrival counters: every CTA of the pair kernel adds 1 to
+  // the counter of its 128 output rows once they are stored (num_n arrivals per band
+  // per launch), so a row consumer can start on a band before the whole GEMM ends.
+  // Only honoured on the pair path (gemm_uses_pair).
+  int* band_flags = nullptr;
 };
 
 zdit_status launch_gemm(const GemmArgs& a, cudaStream_t s);
+bool gemm_uses_pair(int M, int N);
 
 // ---------------------------------------------------------------- attention
 struct AttnArgs {
@@ -108,6 +114,10 @@ struct ResidArgs {
   const float* next_scale;
   int next_scale_stride;
   __nv_bfloat16* next_out;
+  // Optional: instead of waiting for the whole producing GEMM, row t waits until
+  // band_flags[t / 128] >= band_target (that GEMM's counters, see GemmArgs).
+  const int* band_flags = nullptr;
+  int band_target = 0;
 };
 void launch_residual(const ResidArgs& a, cudaStream_t s);
 

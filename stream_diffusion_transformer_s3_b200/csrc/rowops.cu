@@ -158,14 +158,44 @@ struct ResidParams {
   const float* next_scale;
   int next_scale_stride;
   __nv_bfloat16* next_out;
+  const int* band_flags;
+  int band_target;
+  int* err;
 };
 
 template <int MAXV>
 __global__ void __launch_bounds__(RT) residual_kernel(ResidParams p) {
   __shared__ float sh[RT / 32];
-  griddep_wait();
-  griddep_trigger();
+  __shared__ int band_ok;
   const int t = blockIdx.x;
+  if (p.band_flags != nullptr) {
+    // The producing GEMM signals each 128-row band once all its tiles are stored, so
+    // this row starts then instead of after the whole GEMM: the CTAs run beside the
+    // GEMM's last tiles.  Everything else this kernel reads was complete before that
+    // GEMM passed its own dependency wait, which precedes the launch of this grid.
+    if (threadIdx.x == 0) {
+      const int* f = p.band_flags + (t >> 7);
+      const uint64_t t0 = globaltimer_ns();
+      int v;
+      while (true) {
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+        if (v >= p.band_target) break;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+          atomicCAS(p.err, 0, -7 /* ZDIT_ERR_DEVICE_TIMEOUT */);
+          v = -1;
+          break;
+        }
+        __nanosleep(200);
+      }
+      band_ok = v >= 0;
+    }
+    __syncthreads();
+    griddep_trigger();
+    if (!band_ok) return;  // uniform across the CTA
+  } else {
+    griddep_wait();
+    griddep_trigger();
+  }
   const __nv_bfloat16* yr = p.y + (size_t)t * p.D;
   float* xr = p.x + (size_t)t * p.D;
   float4 y[MAXV];
@@ -518,7 +548,8 @@ void launch_norm_modulate(const RowModArgs& a, cudaStream_t s) {
 void launch_residual(const ResidArgs& a, cudaStream_t s) {
   ProfScope ps(PROF_RESIDUAL, 0.0, (double)a.T * a.D * (10.0 + (a.next_out ? 2.0 : 0.0)), s);
   ResidParams p{a.x,       a.y,    a.D,          a.post_w,  a.gate,       a.gate_stride, a.tanh_gate,
-                a.cu_seqlens, a.batch, a.eps,    a.next_w,  a.next_scale, a.next_scale_stride, a.next_out};
+                a.cu_seqlens, a.batch, a.eps,    a.next_w,  a.next_scale, a.next_scale_stride, a.next_out,
+                a.band_flags, a.band_target, device_error_ptr()};
   const int v = (a.D + RT * 4 - 1) / (RT * 4);
   if (a.T <= 0) return;
   if (v <= 1)
