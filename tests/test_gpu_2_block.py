@@ -69,3 +69,19 @@ def test_tiny_block_more_branches(n_caps, n_valids):
     # every branch has its own adaLN vector: covers the batched projection for B = 3 and 8
     case = synth.block_case(7, synth.TINY, 8, 8, n_caps, n_valids)
     _check(case, synth.TINY, O.Flags())
+
+
+def test_band_overlap_is_bitwise_neutral():
+    # After the out and down projections the residual rows normally start band by band
+    # while the projection's last tiles run (counters in the workspace); under the event
+    # profiler every kernel waits for its predecessor instead.  Same bits either way.
+    import stream_diffusion_transformer_s3_b200 as Z
+    case = synth.config2(2)  # full width: T = 608 takes the CTA-pair GEMM path
+    flags = O.Flags()
+    banded = run_block_gpu(case, synth.FULL, flags)
+    Z.zdit_profile_begin(4096)
+    try:
+        serial = run_block_gpu(case, synth.FULL, flags)
+    finally:
+        Z.zdit_profile_end()
+    assert np.array_equal(banded, serial)
