@@ -204,7 +204,8 @@ __global__ void __launch_bounds__(RT) residual_kernel(ResidParams p) {
   for (int i = 0; i < MAXV; ++i) {
     const int idx = (i * RT + threadIdx.x) * 4;
     if (idx < p.D) {
-      const uint2 u = *reinterpret_cast<const uint2*>(yr + idx);
+      // L2 loads: y may have been written by another SM moments ago (band-by-band start)
+      const uint2 u = __ldcg(reinterpret_cast<const uint2*>(yr + idx));
       const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
       const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
       y[i] = make_float4(__low2float(lo), __high2float(lo), __low2float(hi), __high2float(hi));
