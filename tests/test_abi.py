@@ -6,7 +6,6 @@ import os
 import re
 
 import numpy as np
-import pytest
 
 import oracle as O
 import stream_diffusion_transformer_s3_b200 as Z

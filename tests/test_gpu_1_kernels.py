@@ -1,7 +1,6 @@
 """Kernel-level parity on the GPU: projection GEMM, joint attention, RoPE tables,
 the fused negated-CFG Euler update and patchify, each against the CPU oracle (or a
 float64 matrix product for the GEMM) on seeded inputs."""
-import math
 
 import numpy as np
 import pytest

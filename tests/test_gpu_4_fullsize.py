@@ -14,7 +14,7 @@ import torch
 import oracle as O
 import stream_diffusion_transformer_s3_b200 as Z
 from stream_diffusion_transformer_s3_b200 import synth
-from _gpu import BlockSource, LazyBlock, bf16, dev, dims_of, errors, host, require_gpu, run_block_gpu, run_stack
+from _gpu import BlockSource, LazyBlock, bf16, dev, errors, host, require_gpu, run_block_gpu, run_stack
 
 pytestmark = pytest.mark.gpu
 TOL = 2e-2

@@ -8,7 +8,6 @@ workspace, within the block-parity tolerance, and that a call too large for the
 40 MiB scratch is refused before any launch.  This file is collected last."""
 import ctypes as C
 
-import numpy as np
 import pytest
 import torch
 
