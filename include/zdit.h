@@ -172,13 +172,17 @@ ZDIT_API zdit_status zdit_block_forward(const zdit_block_cfg* cfg, const zdit_bl
  *   nothing.  At full width (D 3840, F 10240, two branches) that admits up to 907 tokens,
  *   e.g. the 256px cond/uncond pair (608 tokens, 26.8 MiB).
  *   The call allocates nothing (no cudaMalloc, cudaFree or allocating library call).
- *   The first call on a device looks up the array's device address (once per
- *   device, with that device current); make that first call before any stream
+ *   Every call looks up the array's device address on the current device
+ *   (cudaGetSymbolAddress); the first lookup on a device loads the library's module
+ *   that holds the array, so make the first call on each device before any stream
  *   capture.
- *   All calls share the one array and it keeps the previous call's contents (the
- *   block writes every workspace byte it reads, so nothing needs clearing): calls
- *   whose execution overlaps on the GPU (different streams, or host threads) race
- *   on it and must be serialized by the caller.
+ *   All calls share the one array and it keeps the previous call's contents: the
+ *   block writes every workspace byte it reads, except its per-band arrival
+ *   counters, which each call zeroes on its stream before using them.  Calls whose
+ *   execution overlaps on the GPU (different streams, or host threads) race on the
+ *   array and must be serialized by the caller.
+ *   Arguments are checked in the same order as zdit_block_forward; the size check
+ *   comes after them.
  * Errors: as zdit_block_forward, plus ZDIT_ERR_WORKSPACE (too many tokens) and
  * ZDIT_ERR_CUDA (address lookup failed). */
 ZDIT_API zdit_status zdit_block_forward_static(const zdit_block_cfg* cfg, const zdit_block_weights* w,

@@ -129,7 +129,11 @@ inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) =
 
 // Band counters of one forward: zeroed when the token count changes, then every
 // projection that signals them adds num_n arrivals per band, so the k-th one of the
-// run is complete for a band at k * num_n.
+// run is complete for a band at k * num_n.  A BandState lives for one block or stack
+// call only (T starts at -1), so every call re-zeroes the counters in its workspace
+// before the first projection that signals them: a reused workspace (the static
+// scratch of zdit_block_forward_static included) never carries stale counts into the
+// next call.  Caching a BandState across calls would break that.
 struct BandState {
   int T = -1;
   int epoch = 0;
@@ -470,6 +474,25 @@ zdit_status stack_run(const zdit_stack_cfg* cfg, const zdit_stack_weights* w, co
 }  // namespace
 }  // namespace zdit
 
+namespace zdit {
+
+zdit_status check_block_call(const zdit_block_cfg* cfg, const zdit_block_weights* w, const zdit_varlen* varlen,
+                             const float* x, const float* temb, const float* rope_cos, const float* rope_sin,
+                             const void* workspace, bool with_workspace) {
+  if (!cfg || !w || !varlen || !x || !rope_cos || !rope_sin || (with_workspace && !workspace))
+    return ZDIT_ERR_INVALID_ARG;
+  if (!cfg_ok(cfg) || !varlen_ok(varlen)) return ZDIT_ERR_SHAPE;
+  if (!block_weights_ok(*cfg, *w)) return ZDIT_ERR_INVALID_ARG;
+  if ((cfg->flags & ZDIT_F_ADALN) && !temb) return ZDIT_ERR_INVALID_ARG;
+  if (!al16(x) || !al16(rope_cos) || !al16(rope_sin) ||
+      (with_workspace && (reinterpret_cast<uintptr_t>(workspace) & 255)))
+    return ZDIT_ERR_ALIGNMENT;
+  if (!device_ok()) return ZDIT_ERR_UNSUPPORTED;
+  return ZDIT_OK;
+}
+
+}  // namespace zdit
+
 using namespace zdit;
 
 extern "C" {
@@ -500,13 +523,8 @@ ZDIT_API zdit_status zdit_block_forward(const zdit_block_cfg* cfg, const zdit_bl
                                         const zdit_varlen* varlen, float* x, const float* temb,
                                         const float* rope_cos, const float* rope_sin, void* workspace,
                                         size_t workspace_bytes, void* stream) {
-  if (!cfg || !w || !varlen || !x || !rope_cos || !rope_sin || !workspace) return ZDIT_ERR_INVALID_ARG;
-  if (!cfg_ok(cfg) || !varlen_ok(varlen)) return ZDIT_ERR_SHAPE;
-  if (!block_weights_ok(*cfg, *w)) return ZDIT_ERR_INVALID_ARG;
-  if ((cfg->flags & ZDIT_F_ADALN) && !temb) return ZDIT_ERR_INVALID_ARG;
-  if (!al16(x) || !al16(rope_cos) || !al16(rope_sin) || (reinterpret_cast<uintptr_t>(workspace) & 255))
-    return ZDIT_ERR_ALIGNMENT;
-  if (!device_ok()) return ZDIT_ERR_UNSUPPORTED;
+  const zdit_status v = check_block_call(cfg, w, varlen, x, temb, rope_cos, rope_sin, workspace, true);
+  if (v != ZDIT_OK) return v;
   const int T = varlen->cu_seqlens_host[varlen->batch];
   const size_t need = zdit_block_workspace_bytes(cfg, T, varlen->batch);
   if (workspace_bytes < need) return ZDIT_ERR_WORKSPACE;

@@ -122,6 +122,13 @@ struct ResidArgs {
 void launch_residual(const ResidArgs& a, cudaStream_t s);
 
 
+// Host-side argument checks of one block call, in the order zdit_block_forward runs
+// them (null pointers, cfg and varlen shapes, weights, temb, alignment, device);
+// with_workspace adds the caller workspace (non-null, 256-byte aligned).
+zdit_status check_block_call(const zdit_block_cfg* cfg, const zdit_block_weights* w, const zdit_varlen* varlen,
+                             const float* x, const float* temb, const float* rope_cos, const float* rope_sin,
+                             const void* workspace, bool with_workspace);
+
 int num_sms();
 // true while zdit_profile_begin .. zdit_profile_end is recording
 bool profiling_on();

@@ -11,35 +11,27 @@
 // the process exits.  Calls whose workspace would exceed that are rejected.
 #include <cuda_runtime.h>
 
-#include <mutex>
-
 #include "../../include/zdit.h"
+#include "internal.h"
 
 namespace {
 
 constexpr size_t kStaticScratchBytes = size_t(40) << 20;  // 40 MiB
 
 // The shared scratch.  In host code this name is only a host-side handle of the
-// device variable, never a device address: the address is looked up per device with
-// cudaGetSymbolAddress and passed to the kernels.
+// device variable, never a device address: the address is looked up on the current
+// device with cudaGetSymbolAddress and passed to the kernels.
 static __device__ __align__(256) unsigned char g_block_scratch[kStaticScratchBytes];
 
-constexpr int kMaxDevices = 64;
-
-// Device address of g_block_scratch on the current device, looked up once per device
-// (with that device current) and cached.  nullptr if the lookup fails.
+// Device address of g_block_scratch on the current device, or nullptr if the lookup
+// fails.  Looked up on every call rather than cached: after cudaDeviceReset (or a
+// primary-context release and re-creation) the module is loaded again and the array
+// may sit at another address.  Once the module is loaded the lookup is cheap; the
+// first one on a device loads the module.
 void* scratch_on_current_device() {
-  static std::mutex mu;
-  static void* addr[kMaxDevices] = {};
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_block_scratch) != cudaSuccess) return nullptr;
-    addr[dev] = p;
-  }
-  return addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_block_scratch) != cudaSuccess) return nullptr;
+  return p;
 }
 
 }  // namespace
@@ -48,14 +40,18 @@ extern "C" ZDIT_API zdit_status zdit_block_forward_static(const zdit_block_cfg* 
                                                           const zdit_varlen* varlen, float* x, const float* temb,
                                                           const float* rope_cos, const float* rope_sin,
                                                           void* stream) {
-  if (!cfg || !varlen || !varlen->cu_seqlens_host || varlen->batch <= 0) return ZDIT_ERR_INVALID_ARG;
+  // the same checks, in the same order, as zdit_block_forward (minus the workspace)
+  const zdit_status v = zdit::check_block_call(cfg, w, varlen, x, temb, rope_cos, rope_sin, nullptr, false);
+  if (v != ZDIT_OK) return v;
   const int64_t T = varlen->cu_seqlens_host[varlen->batch];
   const size_t need = zdit_block_workspace_bytes(cfg, T, varlen->batch);
   if (need == 0) return ZDIT_ERR_SHAPE;
   if (need > kStaticScratchBytes) return ZDIT_ERR_WORKSPACE;  // too many tokens for the static scratch
   void* scratch = scratch_on_current_device();
   if (scratch == nullptr) return ZDIT_ERR_CUDA;
-  // Every workspace region of the block is fully written before it is read, so the
-  // scratch needs no clearing between calls.
+  // Every workspace region is written before it is read within a call, except the
+  // per-band arrival counters of the out and down projections: those are zeroed by the
+  // block's launch sequence at the start of each call (its band state lives for one call
+  // only), so the previous call's contents never leak into this one.
   return zdit_block_forward(cfg, w, varlen, x, temb, rope_cos, rope_sin, scratch, kStaticScratchBytes, stream);
 }

@@ -4,8 +4,9 @@ own pool, or a loop that must not pay cudaMalloc's device-wide synchronization).
 
 Checks, through the C ABI on the GPU, that two calls in a row (sharing the library's
 static scratch) give the same block output as zdit_block_forward with a caller
-workspace, within the block-parity tolerance, and that a call too large for the
-40 MiB scratch is refused before any launch.  This file is collected last."""
+workspace, within the block-parity tolerance; that those two calls leave the device's
+free memory unchanged (they allocate nothing); and that a call too large for the 40 MiB
+scratch is refused before any launch.  This file is collected last."""
 import ctypes as C
 
 import pytest
@@ -41,10 +42,23 @@ def test_static_scratch_block_matches_workspace_block_twice():
     ref = host(x_ref)
     upd_ref = ref - case["x"]
 
-    for _ in range(2):  # the second call finds the first call's data in the scratch
-        x = dev(case["x"])
+    # every device buffer of the measured calls exists before the free-memory reading;
+    # one warm-up call loads the module that holds the scratch array
+    x0 = dev(case["x"])
+    xs = [torch.empty_like(x0) for _ in range(3)]
+    xs[2].copy_(x0)
+    Z.zdit_block_forward_static(dims, fl, w, vl, xs[2], temb, cs, sn)
+    assert Z.zdit_device_status() == 0
+    torch.cuda.synchronize()
+    free_before = torch.cuda.mem_get_info()[0]
+    for x in xs[:2]:  # the second call finds the first call's data in the scratch
+        x.copy_(x0)
         Z.zdit_block_forward_static(dims, fl, w, vl, x, temb, cs, sn)
         assert Z.zdit_device_status() == 0
+    torch.cuda.synchronize()
+    free_after = torch.cuda.mem_get_info()[0]
+    assert free_after == free_before, (free_before, free_after)
+    for x in xs[:2]:
         got = host(x)
         e_out = errors(got, ref)
         e_upd = errors(got - case["x"], upd_ref)
