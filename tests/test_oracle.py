@@ -209,6 +209,8 @@ def _torch_block(d, case, flags):
     if flags.adaln:
         mod = torch.nn.functional.linear(temb, w["w_ada"], w["b_ada"])
         s1, g1, s2, g2 = mod.chunk(4, dim=1)
+        if flags.tanh_gate:  # only the two gate chunks pass through tanh; the scales do not
+            g1, g2 = torch.tanh(g1), torch.tanh(g2)
     else:
         s1 = s2 = torch.zeros(len(cu) - 1, D, dtype=torch.float64)
         g1 = g2 = torch.ones(len(cu) - 1, D, dtype=torch.float64)
@@ -246,7 +248,8 @@ def _torch_block(d, case, flags):
 
 
 @pytest.mark.parametrize("flags", [O.Flags(), O.Flags(sandwich=False),
-                                   O.Flags(qk_norm=True), O.Flags(adaln=False)])
+                                   O.Flags(qk_norm=True), O.Flags(adaln=False),
+                                   O.Flags(tanh_gate=True), O.Flags(tanh_gate=True, sandwich=False)])
 def test_block_matches_torch_composition(flags):
     d, case = _tiny_case(adaln=flags.adaln, qk_norm=flags.qk_norm, n_caps=(32, 64),
                          n_valids=(25, 40))
@@ -384,6 +387,38 @@ def test_timestep_embedding_at_zero():
     emb = O.timestep_embedding(np.array([0.0]), w)
     np.testing.assert_allclose(emb[0, :128], O.silu(np.ones(128)), rtol=1e-15)
     np.testing.assert_allclose(emb[0, 128:], 0.0, atol=0)
+
+
+def test_timestep_embedding_frequencies_at_nonzero_t():
+    # Reading of the timestep embedding: the first half holds cos and the second half sin
+    # of 1000 t times frequencies spaced geometrically from 1 down to 10000^(-127/128).
+    # With identity MLP weights and zero biases the output is silu(embedding); the
+    # expected values are written as a scalar loop with 10000 ** (-i / 128), another
+    # expression than the oracle's exp(-ln(10000) i / half), so a divisor of (half - 1),
+    # swapped cos / sin halves or a wrong time scale each fail here.
+    w = {"w_t1": np.eye(256), "b_t1": np.zeros(256), "w_t2": np.eye(256), "b_t2": np.zeros(256)}
+    t = 0.37
+    emb = O.timestep_embedding(np.array([t]), w)[0]
+    silu = lambda v: v / (1.0 + math.exp(-v))
+    expect = [silu(math.cos(1000.0 * t * 10000.0 ** (-i / 128))) for i in range(128)]
+    expect += [silu(math.sin(1000.0 * t * 10000.0 ** (-i / 128))) for i in range(128)]
+    np.testing.assert_allclose(emb, np.array(expect), rtol=1e-12, atol=1e-12)
+    # two entries worked by hand: i = 0 -> argument 370 rad; i = 64 -> 370 / 100 = 3.7 rad
+    assert emb[0] == pytest.approx(silu(math.cos(370.0)), abs=1e-12)
+    assert emb[128 + 64] == pytest.approx(silu(math.sin(3.7)), abs=1e-12)
+
+
+def test_tanh_gate_touches_only_the_gate_chunks():
+    # adaLN with the tanh-gate option: chunks (scale_attn, gate_attn, scale_ffn, gate_ffn);
+    # only the gates pass through tanh.  Checked on a hand-set projection whose output
+    # chunks are known: bias only, chunk c filled with the value c + 0.5.
+    D, E = 4, 8
+    w = {"w_ada": np.zeros((4 * D, E)), "b_ada": np.repeat(np.arange(4) + 0.5, D)}
+    s1, g1, s2, g2 = O.adaln_vectors(np.ones((1, E)), w, D, O.Flags(tanh_gate=True))
+    np.testing.assert_array_equal(s1, np.full((1, D), 0.5))
+    np.testing.assert_allclose(g1, np.full((1, D), math.tanh(1.5)), rtol=1e-15)
+    np.testing.assert_array_equal(s2, np.full((1, D), 2.5))
+    np.testing.assert_allclose(g2, np.full((1, D), math.tanh(3.5)), rtol=1e-15)
 
 
 def test_fp16_cannot_hold_projection_outputs():
