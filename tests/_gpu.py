@@ -27,6 +27,15 @@ def host(t):
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
+from _parity import ParityError, assert_parity, parity_metrics  # noqa: F401  (re-exported)
+
+# bf16 roundings on the block path, for the element bound of assert_parity: the
+# operands a, q, k, v, P, o, a2, h and the stored projection outputs y (twice)
+N_ROUND_BLOCK = 10
+# attention alone: P before the PV product and the stored output
+N_ROUND_ATTN = 2
+
+
 def errors(got, ref):
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)

@@ -1,15 +1,15 @@
 """Block-level parity on the GPU: zdit_block_forward against the oracle's
 block_forward on the tiny single-block case and the full-width cond/uncond pair.
 
-Tolerance: relative L2 error <= 2e-2 on the block output and, more strictly, on
-the block's update (output minus input); mean and median absolute errors are
-reported alongside."""
+Tolerance: relative L2 error <= 2e-2 on the block output and on the block's update
+(output minus input), and on the update per token row and per element (tests/_parity.py);
+mean and median absolute errors are reported alongside."""
 import numpy as np
 import pytest
 
 import oracle as O
 from stream_diffusion_transformer_s3_b200 import synth
-from _gpu import errors, require_gpu, run_block_gpu
+from _gpu import N_ROUND_BLOCK, assert_parity, require_gpu, run_block_gpu
 
 pytestmark = pytest.mark.gpu
 TOL = 2e-2
@@ -24,13 +24,7 @@ def _check(case, d, flags):
     got = run_block_gpu(case, d, flags)
     ref = O.block_forward(case["x"], case["cu_seqlens"], case["pos"], case["temb"], case["weights"], d, flags)
     x0 = case["x"].astype(np.float64)
-    e_out = errors(got, ref)
-    e_upd = errors(got - x0, ref - x0)
-    print(f"\n{flags}: out {e_out}\n  update {e_upd}")
-    assert np.all(np.isfinite(got))
-    assert e_out["rel_l2"] <= TOL, e_out
-    assert e_upd["rel_l2"] <= TOL, e_upd
-    return e_upd
+    return assert_parity(got, ref, TOL, base=x0, n_round=N_ROUND_BLOCK, label=str(flags))
 
 
 @pytest.mark.parametrize("flags", [

@@ -4,7 +4,7 @@ import pytest
 
 import oracle as O
 from stream_diffusion_transformer_s3_b200 import synth
-from _gpu import BlockSource, LazyBlock, errors, require_gpu, run_stack
+from _gpu import N_ROUND_BLOCK, BlockSource, LazyBlock, assert_parity, require_gpu, run_stack
 
 pytestmark = pytest.mark.gpu
 
@@ -21,9 +21,7 @@ def test_small_stack_matches_oracle(n_caps, n_valids):
     case = synth.stack_case(7, 8, 8, list(n_caps), list(n_valids), [0.4] * len(n_caps), cap_dim=128)
     got = run_stack(W, case, d, 1, 1, 2, 128)
     ref = O.stack_forward(case, W, d)
-    e = errors(got, ref)
-    print("\nstack", e)
-    assert e["rel_l2"] <= 2e-2, e
+    assert_parity(got, ref, 2e-2, n_round=N_ROUND_BLOCK, label=f"stack {n_caps}")
 
 
 def test_full_width_stack_two_blocks_per_kind_256px():
@@ -33,9 +31,7 @@ def test_full_width_stack_two_blocks_per_kind_256px():
     case = synth.stack_case(3, 16, 16, [64, 32], [45, 1], [0.25, 0.25])
     got = run_stack(W, case, d, 1, 1, 1, 2560)
     ref = O.stack_forward(case, W, d)
-    e = errors(got, ref)
-    print("\nstack full width", e)
-    assert e["rel_l2"] <= 2e-2, e
+    assert_parity(got, ref, 2e-2, n_round=N_ROUND_BLOCK, label="stack full width")
 
 
 def test_full_width_full_depth_stack_256px():
@@ -52,7 +48,5 @@ def test_full_width_full_depth_stack_256px():
     ref = O.stack_forward(case, dict(W, blocks=[LazyBlock(src, i) for i in range(len(kinds))], block_kinds=kinds), d)
     assert all(b is not None for b in src.device)
     got = run_stack(W, case, d, 2, 2, 30, 2560, blocks=src.device)
-    e = errors(got, ref)
-    print("\nstack full width, 34 blocks", e)
     # per-block bound 2e-2; the measured 34-block free-running error is 4.9e-3
-    assert e["rel_l2"] <= 2e-2, e
+    assert_parity(got, ref, 2e-2, n_round=N_ROUND_BLOCK, label="stack full width, 34 blocks")

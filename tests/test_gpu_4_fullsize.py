@@ -1,10 +1,12 @@
 """Parity at the full sizes of the 1024x1024 workload, in the launch configuration
 bench.py times: one main block over the joint cond/uncond sequence (4224 + 4128
-tokens, width 3840) checked on sampled rows against the oracle; the attention-only
-sweep sizes checked on sampled query rows; the whole 34-block stack checked through
-properties that hold at any size (branch isolation, determinism, finiteness) and, on request
-(ZDIT_FULL_STACK_PARITY=1: the float64 oracle of the whole forward takes minutes of host
-time), free-running against the oracle."""
+tokens, width 3840) and one noise-refiner block over the image tokens of both branches
+(2 x 4096 tokens) checked on sampled rows against the oracle (teacher-forced); the
+attention-only sweep sizes checked on sampled query rows; the whole 34-block forward
+free-running against the oracle's output of the same seeded inputs (stored by
+tests/golden/make_stack_1024.py, since the float64 forward takes a quarter of an hour of
+host time), and through properties that hold at any size (branch isolation,
+determinism)."""
 import os
 
 import numpy as np
@@ -14,7 +16,8 @@ import torch
 import oracle as O
 import stream_diffusion_transformer_s3_b200 as Z
 from stream_diffusion_transformer_s3_b200 import synth
-from _gpu import BlockSource, LazyBlock, bf16, dev, errors, host, require_gpu, run_block_gpu, run_stack
+from _gpu import (N_ROUND_ATTN, N_ROUND_BLOCK, BlockSource, assert_parity, bf16, dev, host, require_gpu,
+                  run_block_gpu, run_stack)
 
 pytestmark = pytest.mark.gpu
 TOL = 2e-2
@@ -47,11 +50,26 @@ def test_fullsize_main_block_sampled_rows():
     ref = O.block_forward_rows(case["x"], case["cu_seqlens"], case["pos"], case["temb"], case["weights"], d,
                                rows, O.Flags())
     x0 = case["x"][rows].astype(np.float64)
-    e_upd = errors(got[rows] - x0, ref - x0)
-    e_out = errors(got[rows], ref)
-    print(f"\nfull-size block, {len(rows)} rows: update {e_upd}")
-    assert e_upd["rel_l2"] <= TOL, e_upd
-    assert e_out["rel_l2"] <= TOL, e_out
+    assert_parity(got[rows], ref, TOL, base=x0, n_round=N_ROUND_BLOCK,
+                  label=f"full-size main block, {len(rows)} sampled rows")
+
+
+def test_fullsize_noise_refiner_block_sampled_rows():
+    # a noise-refiner block at its real size: the image tokens of both branches (2 x 4096,
+    # 64 x 64 grid each) as two segments, adaLN, image positions (n_cap_b + 1, h, w) with
+    # the branches' caption lengths 128 and 32
+    d = synth.FULL
+    seed = 23
+    n_img = 64 * 64
+    cu = synth.cu_seqlens([n_img, n_img])
+    pos = np.concatenate([synth.branch_positions(64, 64, c)[:n_img] for c in (128, 32)])
+    case = {"x": synth.randn(seed, 1, (2 * n_img, d.dim)), "cu_seqlens": cu, "pos": pos,
+            "temb": synth.randn(seed, 2, (2, d.temb_dim)), "weights": synth.block_weights(seed, 0, d)}
+    got = run_block_gpu(case, d, O.Flags())
+    rows = _sample_rows(cu, 2)
+    ref = O.block_forward_rows(case["x"], cu, pos, case["temb"], case["weights"], d, rows, O.Flags())
+    assert_parity(got[rows], ref, TOL, base=case["x"][rows].astype(np.float64), n_round=N_ROUND_BLOCK,
+                  label=f"full-size noise-refiner block, {len(rows)} sampled rows")
 
 
 @pytest.mark.parametrize("n_img,n_cap", [(1024, 32), (4096, 128), (16384, 512)])
@@ -74,9 +92,7 @@ def test_attention_sweep_sampled_rows(n_img, n_cap):
         for h in range(H):
             sl = slice(h * 128, (h + 1) * 128)
             ref[i, sl] = O.softmax_attention(c["q"][r:r + 1, sl], c["k"][s:e, sl], c["v"][s:e, sl])[0]
-    e = errors(got[rows], ref)
-    print(f"\nattention {lengths}: {e}")
-    assert e["rel_l2"] <= 1e-2, e
+    assert_parity(got[rows], ref, 1e-2, n_round=N_ROUND_ATTN, label=f"attention {lengths}, {len(rows)} sampled rows")
 
 
 def _device_stack(seed=77):
@@ -130,20 +146,23 @@ def test_fullsize_stack_branch_isolation_and_determinism():
     assert (both[0] - both[1]).abs().max().item() > 1e-3
 
 
-@pytest.mark.skipif(os.environ.get("ZDIT_FULL_STACK_PARITY") != "1",
-                    reason="the float64 oracle of the whole 1024x1024 forward takes ~7 min of host time")
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "stack_1024_seed31.npz")
+
+
 def test_fullsize_stack_free_running():
-    # the benchmarked workload end to end: 64x64 image grid per branch, captions 128 (100 valid)
-    # and 32 (1 valid), 2 + 2 + 30 full-width blocks, embedders and final layer, against the
-    # oracle's stack_forward on the same inputs
+    # the benchmarked workload end to end, free-running: 64x64 image grid per branch,
+    # captions 128 (100 valid) and 32 (1 valid), 2 + 2 + 30 full-width blocks, embedders
+    # and final layer, against the oracle's stack_forward of the same seeded inputs
+    g = np.load(GOLDEN)
+    seed = int(g["seed"])
     d = synth.FULL
-    seed = 31
-    kinds = ["noise"] * 2 + ["context"] * 2 + ["main"] * 30
+    kinds = [str(k) for k in g["kinds"]]
     W = synth.stack_weights(seed, d, blocks=False)
     src = BlockSource(seed, d, kinds)
-    case = synth.stack_case(seed, 64, 64, [128, 32], [100, 1], [0.5, 0.5])
-    ref = O.stack_forward(case, dict(W, blocks=[LazyBlock(src, i) for i in range(len(kinds))], block_kinds=kinds), d)
+    for i in range(len(kinds)):  # draws each block once and uploads it
+        src.host(i)
+    case = synth.stack_case(seed, int(g["grid"][0]), int(g["grid"][1]), [int(c) for c in g["n_caps"]],
+                            [int(v) for v in g["n_valids"]], [float(t) for t in g["t"]])
     got = run_stack(W, case, d, 2, 2, 30, 2560, blocks=src.device)
-    e = errors(got, ref)
-    print("\nstack 1024x1024, 34 blocks, free-running", e)
-    assert e["rel_l2"] <= TOL, e
+    ref = g["out"].astype(np.float64)
+    assert_parity(got, ref, TOL, n_round=N_ROUND_BLOCK, label="1024x1024 forward, 34 blocks, free-running")

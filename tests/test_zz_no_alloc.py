@@ -14,7 +14,7 @@ import torch
 
 import stream_diffusion_transformer_s3_b200 as Z
 from stream_diffusion_transformer_s3_b200 import synth
-from _gpu import dev, dims_of, errors, host, require_gpu, rope_tables
+from _gpu import N_ROUND_BLOCK, assert_parity, dev, dims_of, host, require_gpu, rope_tables
 
 pytestmark = pytest.mark.gpu
 TOL = 2e-2
@@ -40,7 +40,6 @@ def test_static_scratch_block_matches_workspace_block_twice():
     Z.zdit_block_forward(dims, fl, w, vl, x_ref, temb, cs, sn, ws)
     assert Z.zdit_device_status() == 0
     ref = host(x_ref)
-    upd_ref = ref - case["x"]
 
     # every device buffer of the measured calls exists before the free-memory reading;
     # one warm-up call loads the module that holds the scratch array
@@ -58,12 +57,8 @@ def test_static_scratch_block_matches_workspace_block_twice():
     torch.cuda.synchronize()
     free_after = torch.cuda.mem_get_info()[0]
     assert free_after == free_before, (free_before, free_after)
-    for x in xs[:2]:
-        got = host(x)
-        e_out = errors(got, ref)
-        e_upd = errors(got - case["x"], upd_ref)
-        assert e_out["rel_l2"] <= TOL, e_out
-        assert e_upd["rel_l2"] <= TOL, e_upd
+    for i, x in enumerate(xs[:2]):
+        assert_parity(host(x), ref, TOL, base=case["x"], n_round=N_ROUND_BLOCK, label=f"static scratch, call {i + 1}")
 
 
 def test_static_scratch_refuses_oversized_call():
