@@ -54,9 +54,10 @@ def forward_flops() -> float:
 
 
 # DRAM bytes per launch of the dominant kernel (gate/up GEMM of a main block, 8352 x 20480
-# x 3840), from one ncu capture (profiles/gemm_gate_up_swiglu_block_1024.md), valid for the
-# GEMM sources with this hash only; any change to them makes the figure stale (reported null).
-NCU_TRAFFIC = {"kernel": "gemm_gate_up_swiglu", "bytes": 409049600 + 156176384, "src_hash": "7a8075dead156cf5"}
+# x 3840), from one ncu capture of that kernel (dram__bytes_read.sum + dram__bytes_write.sum),
+# valid for the GEMM sources with this hash only; any change to them makes the figure stale
+# (reported null).
+NCU_TRAFFIC = {"kernel": "gemm_gate_up_swiglu", "bytes": 409473536 + 156275456, "src_hash": "b057c4233dacc1b0"}
 
 
 def gemm_src_hash() -> str:
@@ -138,6 +139,12 @@ SAMPLER_WORKLOAD = ("1024x1024 image: 8-step FlowMatchEuler sampler with negated
                     "cond/uncond pair, 34-block DiT, caption stream computed once (t-independent)")
 BLOCK_WORKLOAD = ("one main DiT block of the 1024x1024 workload: joint cond/uncond sequence 4224 + 4128 "
                   "tokens, width 3840, 30x128 heads, SwiGLU 10240, adaLN + sandwich norm")
+
+
+HBM_WORKLOAD = ("the HBM-bound small kernels of one 1024x1024 step at their real sizes: the adaLN projections "
+                "of the 32 adaLN blocks in one launch (32 x bf16 [15360, 256], cond/uncond temb), the RoPE "
+                "cos/sin tables of the joint sequence (8352 tokens x 64 pairs) and the fused negated-CFG Euler "
+                "update of the 16 x 128 x 128 latent")
 
 
 ATTN_SWEEP_IMG = (1024, 4096, 9216, 16384)
@@ -283,6 +290,33 @@ def run_ours(args):
             latent.copy_(latent0)
             Z.zdit_sample(stack, call, latent, ws, n_steps=8, guidance=1.0, cache_context=True,
                           dedup_noise=args.dedup, use_graph=args.graph)
+    elif args.workload == "hbm":
+        # the small bandwidth-bound kernels of one step at their real sizes; the adaLN
+        # weights (251.7 MB) exceed L2, the tables and the latent are the step's own sizes
+        from stream_diffusion_transformer_s3_b200 import synth
+        n_blk = sum(1 for k in KINDS if k != "context")
+        w_ada = [(torch.randn(4 * D, E, generator=g) * 0.02).to(device=device, dtype=torch.bfloat16)
+                 for _ in range(n_blk)]
+        b_ada = [torch.randn(4 * D, generator=g).to(device) * 0.02 for _ in range(n_blk)]
+        mods = [torch.empty(2, 4 * D, device=device) for _ in range(n_blk)]
+        temb = torch.randn(2, E, generator=g).to(device)
+        pos = torch.from_numpy(synth.joint_positions(GRID[0], GRID[1], list(N_CAPS))).to(device)
+        T = pos.shape[0]
+        cs = torch.empty(T, HD // 2, device=device)
+        sn = torch.empty_like(cs)
+        dims = Z.Dims()
+        z = torch.randn(n_img, PATCH, generator=g).to(device)
+        vel = torch.randn(2, n_img, PATCH, generator=g).to(device)
+        sig = Z.zdit_sigma_schedule(8)
+        inputs, result = [temb, z], z
+        flops = 0.0
+        hbm_bytes = (n_blk * (4 * D * E * 2 + 4 * D * 4 + 2 * 4 * D * 4) + T * (12 + 2 * 4 * HD // 2)
+                     + n_img * PATCH * 16)
+
+        def step(i):
+            Z.zdit_adaln_project(w_ada, b_ada, mods, temb)
+            Z.zdit_rope_table(pos, dims.rope_axes, dims.rope_theta, cs, sn)
+            Z.zdit_euler_cfg_step(z, vel[0], vel[1], 1.0, sig[i % 8], sig[i % 8 + 1])
     else:
         # one main block of the workload: the joint cond/uncond sequence (4224 + 4128)
         from stream_diffusion_transformer_s3_b200 import synth
@@ -377,7 +411,17 @@ def run_ours(args):
     peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
     dom = max(kernels.items(), key=lambda kv: kv[1]["total_ms"]) if kernels else None
     roofline = None
-    if dom is not None:
+    if dom is not None and args.workload == "hbm":
+        name, k = dom
+        achieved = k["bytes"] / (k["total_ms"] * 1e-3) / 1e9
+        roofline = {"kernel": name, "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                    "peak_source": f"{peak_src} copy bandwidth", "traffic": args.traffic,
+                    "launches_per_step": k["launches"] / args.steps,
+                    "ms_per_launch": k["total_ms"] / k["launches"],
+                    "timing": "CUDA events around each launch, in a pass of the same steps right "
+                              "after the timed one"}
+    elif dom is not None:
         name, k = dom
         if k["flops"] > 0:
             achieved = k["flops"] / (k["total_ms"] * 1e-3) / 1e12
@@ -409,7 +453,8 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": {"stack": WORKLOAD, "block": BLOCK_WORKLOAD,
-                                    "sampler": SAMPLER_WORKLOAD, "attention": ATTN_WORKLOAD}[args.workload],
+                                    "sampler": SAMPLER_WORKLOAD, "attention": ATTN_WORKLOAD,
+                                    "hbm": HBM_WORKLOAD}[args.workload],
                        "global_batch": 2 * world, "seq_len": [n_img + c for c in N_CAPS],
                        "flops_per_forward": flops, "parallelism": f"replicas x{world}",
                        "l2": ("working set larger than L2 (12.3 GB of bf16 weights streamed per step)" if args.workload == "stack" else "working set larger than L2 (354 MB weights + 128 MB residual + 448 MB activations per block)"),
@@ -422,6 +467,18 @@ def run_ours(args):
                     "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in h_in),
                     "d2h_bytes_per_step": h_out.numel() * h_out.element_size()},
         }
+        if args.workload == "hbm":
+            res["metric"] = "HBM-bound kernels of the 1024^2 step: algorithmic GB/s (1 B200)"
+            res["value"] = round(world * hbm_bytes / (ms * 1e-3) / 1e9, 1)
+            res["unit"] = "GB/s"
+            res["dtype"] = "f32 / bf16 weights"
+            res["config"]["bytes_per_step"] = hbm_bytes
+            res["config"]["l2"] = ("adaLN weights (251.7 MB) larger than L2; the tables and the latent are the "
+                                   "step's own few MB and stay L2-resident, as in the step")
+            res["e2e"] = {"value": round(world * hbm_bytes / (ms_e2e * 1e-3) / 1e9, 1), "unit": "GB/s",
+                          "ms_per_step": round(ms_e2e, 3), "h2d_bytes_per_step": res["e2e"]["h2d_bytes_per_step"],
+                          "d2h_bytes_per_step": res["e2e"]["d2h_bytes_per_step"]}
+            res["config"].pop("frac_of_peak", None)
         if args.workload == "block":
             res["metric"] = "DiT main-block forward TFLOP/s (1024^2 cond/uncond sequence, bf16, 1 B200)"
         if args.workload == "attention":
@@ -443,6 +500,7 @@ def run_ours(args):
                                          + (", captured as one CUDA graph and replayed" if args.graph else ""))
         if world == 1 and not args.no_cpu_baseline:
             res["cpu_baseline"] = (cpu_baseline_attention() if args.workload == "attention"
+                                   else cpu_baseline_hbm() if args.workload == "hbm"
                                    else cpu_baseline_block(seconds=None))
         print(json.dumps(res), flush=True)
     if world > 1:
@@ -481,6 +539,34 @@ def cpu_baseline_block(seconds=None):
     return {"value": round(flops / dt / 1e12, 5), "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
             "sample": f"one full-width main block of the workload on its uncond branch (L=4128 tokens), "
                       f"NumPy float64 oracle, {dt:.1f} s"}
+
+
+def cpu_baseline_hbm():
+    """The oracle's steps behind the hbm workload on its full sizes: the adaLN vectors of the
+    32 adaLN blocks, the rotary angles (cos / sin) of the joint sequence, the negated-CFG
+    Euler update of the latent; algorithmic bytes of the GPU kernels over the oracle's time."""
+    import numpy as np
+    import oracle as O
+    from stream_diffusion_transformer_s3_b200 import synth
+    n_blk = sum(1 for k in KINDS if k != "context")
+    temb = synth.randn(5, 1, (2, E))
+    ws = [{"w_ada": synth.bf16_round(synth.randn(5, 10 + i, (4 * D, E), 0.02)), "b_ada": synth.randn(5, 100 + i, (4 * D,))}
+          for i in range(n_blk)]
+    pos = synth.joint_positions(GRID[0], GRID[1], list(N_CAPS))
+    n = GRID[0] * GRID[1] * PATCH
+    x, vp, vn = (synth.randn(5, 200 + i, (n,)) for i in range(3))
+    t0 = time.perf_counter()
+    for w in ws:
+        O.adaln_vectors(temb, w, D, O.Flags())
+    phi = O.rope_angles(pos)
+    np.cos(phi), np.sin(phi)
+    O.euler_step(x, O.cfg_velocity(vp, vn, 1.0), 1.0, 0.95)
+    dt = time.perf_counter() - t0
+    T = pos.shape[0]
+    nbytes = n_blk * (4 * D * E * 2 + 4 * D * 4 + 2 * 4 * D * 4) + T * (12 + 2 * 4 * HD // 2) + n * 16
+    return {"value": round(nbytes / dt / 1e9, 2), "unit": "GB/s", "cores": _cores(), "kind": "oracle",
+            "sample": f"the whole hbm workload once (32 adaLN projections, the joint RoPE angles, one "
+                      f"CFG-Euler update), NumPy float64 oracle, {dt:.2f} s"}
 
 
 def cpu_baseline_attention():
@@ -534,10 +620,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["stack", "block", "sampler", "attention"], default="stack",
+    ap.add_argument("--workload", choices=["stack", "block", "sampler", "attention", "hbm"], default="stack",
                     help="stack: the full DiT step (default); block: one main block (for kernel captures); "
                          "sampler: one whole 8-step image per step; attention: joint attention alone at "
-                         "16384 image tokens, with a sweep over sequence lengths")
+                         "16384 image tokens, with a sweep over sequence lengths; hbm: the bandwidth-bound "
+                         "small kernels of one step (adaLN projections, RoPE tables, CFG-Euler)")
     ap.add_argument("--graph", action="store_true",
                     help="sampler workload: the whole image as one captured CUDA graph, replayed")
     ap.add_argument("--dedup", action="store_true",

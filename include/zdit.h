@@ -35,8 +35,14 @@
  *     Device pointers handed to GEMMs or attention must be 16-byte aligned and
  *     their row strides multiples of 8 elements (TMA requirement).
  *   - fp16 is never used: activations reach 3.1e5 ([CoreAI] "fp16 does not work").
- *   - A wait inside a kernel that exceeds 2 s abandons the kernel and latches
- *     ZDIT_ERR_DEVICE_TIMEOUT, reported by zdit_device_status.
+ *   - Every wait inside a kernel (a pipeline barrier, or a row waiting for its
+ *     band of a projection) is bounded: one that exceeds the wait limit abandons
+ *     the kernel and latches ZDIT_ERR_DEVICE_TIMEOUT, reported by
+ *     zdit_device_status.  The limit is fixed when the library is built
+ *     (ZDIT_WAIT_LIMIT_MS, default 2000 ms), one value for every wait: no wait of a
+ *     healthy launch comes near it, but a run that is slowed down from outside (a
+ *     profiler replaying kernels, a debugger, a GPU shared with a heavy job) could
+ *     trip it; build with a larger ZDIT_WAIT_LIMIT_MS for such uses.
  */
 #ifndef ZDIT_H_
 #define ZDIT_H_
@@ -308,8 +314,10 @@ ZDIT_API zdit_status zdit_sigma_schedule(int32_t n_steps, float* sigmas);
  * angle = pos[t, a] * theta^(-2 j / rope_axes[a]), where a is the axis of pair i
  * (pairs [0, axes0/2) -> axis 0, next axes1/2 -> axis 1, rest -> axis 2) and j the
  * pair index inside that axis.  pos: device int32 [T, 3]; cos_out, sin_out:
- * device fp32 [T, head_dim / 2].  [CoreAI] DiT row (3-axis RoPE, precomputed
- * cos/sin).  Errors: ZDIT_ERR_INVALID_ARG, ZDIT_ERR_SHAPE. */
+ * device fp32 [T, head_dim / 2]; head_dim even, at most 1024.  Angles and their
+ * cos / sin are computed in double precision and rounded to fp32.  [CoreAI] DiT
+ * row (3-axis RoPE, precomputed cos/sin).  Errors: ZDIT_ERR_INVALID_ARG,
+ * ZDIT_ERR_SHAPE. */
 ZDIT_API zdit_status zdit_rope_table(const int32_t* pos, int64_t T, int32_t head_dim, const int32_t rope_axes[3],
                                      float theta, float* cos_out, float* sin_out, void* stream);
 
@@ -321,6 +329,24 @@ ZDIT_API zdit_status zdit_rope_table(const int32_t* pos, int64_t T, int32_t head
 ZDIT_API zdit_status zdit_joint_attention(const void* q, int32_t ldq, const void* k, int32_t ldk, const void* v,
                                           int32_t ldv, void* o, int32_t ldo, const zdit_varlen* varlen,
                                           int32_t n_heads, int32_t head_dim, void* stream);
+
+/* The adaLN projections of several blocks in one launch (the first step of every block
+ * with ADALN; zdit_stack_forward computes all of a forward's at once):
+ *   out_i[b, r] = sum_e w_ada_i[r, e] temb[b, e] + b_ada_i[r],  i < n_mat
+ * [CoreAI] DiT row (adaLN in the refiners and main blocks); [Jobs] "Recipes and
+ * precision" (adaLN scaling in FP32).  Each out_i holds the four D-wide chunks
+ * (scale_attn, gate_attn, scale_ffn, gate_ffn) of one block when rows = 4D.
+ *   w_ada    host array of n_mat device pointers, each bf16 [rows, temb_dim], 16-byte aligned
+ *   b_ada    host array of n_mat device pointers, each fp32 [rows]; the array or an entry may
+ *            be NULL (no bias)
+ *   out      host array of n_mat device pointers, each fp32 [batch, rows]
+ *   temb     device fp32 [batch, temb_dim], 16-byte aligned
+ *   n_mat 1..256, batch 1..8, temb_dim a multiple of 8 up to 1024, rows >= 1.
+ * The weights are streamed once (HBM-bound); accumulation in FP32.
+ * Errors: ZDIT_ERR_INVALID_ARG (null pointers), ZDIT_ERR_SHAPE, ZDIT_ERR_ALIGNMENT. */
+ZDIT_API zdit_status zdit_adaln_project(const void* const* w_ada, const float* const* b_ada, float* const* out,
+                                        int32_t n_mat, const float* temb, int32_t batch, int32_t temb_dim,
+                                        int32_t rows, void* stream);
 
 /* Projection GEMM alone: C[M, N] (fp32, row stride ldc) = A[M, K] . B[N, K]^T
  * (+ bias[N] if non-NULL); A, B device bf16 row-major.  The tensor-core kernel
@@ -365,12 +391,17 @@ ZDIT_API int64_t zdit_launch_count(void);
 
 /* Synchronizes `stream`, then returns (and clears) the first device-side error
  * latched by any kernel of this library (ZDIT_ERR_DEVICE_TIMEOUT), or
- * ZDIT_ERR_CUDA if the stream reports a CUDA error, else ZDIT_OK. */
+ * ZDIT_ERR_CUDA if the stream reports a CUDA error, else ZDIT_OK.
+ * The latched error lives in one word per device, shared by every stream and host
+ * thread that uses the library on that device: it reports an error of any of their
+ * launches, not only of `stream`'s, and reading it clears it for all of them.  Callers
+ * that run the library on several streams of one device at once must coordinate who
+ * reads it. */
 ZDIT_API zdit_status zdit_device_status(void* stream);
 
 /* Health check of the bounded waits used by every pipelined kernel: launches one
  * kernel that waits on a barrier nothing arrives on; after the library's wait limit
- * (2 s) it gives up, latches ZDIT_ERR_DEVICE_TIMEOUT (read with
+ * (ZDIT_WAIT_LIMIT_MS, 2 s by default) it gives up, latches ZDIT_ERR_DEVICE_TIMEOUT (read with
  * zdit_device_status) and writes 2 to *result_dev (device int32; 1 would mean the
  * wait wrongly succeeded).  The context stays usable.  Not part of the DiT path.
  * Errors: ZDIT_ERR_INVALID_ARG, ZDIT_ERR_CUDA. */

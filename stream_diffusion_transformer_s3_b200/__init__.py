@@ -102,6 +102,8 @@ _SIGS = {
     "zdit_joint_attention": (C.c_int, [C.c_void_p, C.c_int32, C.c_void_p, C.c_int32, C.c_void_p,
                                        C.c_int32, C.c_void_p, C.c_int32, C.POINTER(Varlen), C.c_int32,
                                        C.c_int32, C.c_void_p]),
+    "zdit_adaln_project": (C.c_int, [C.POINTER(C.c_void_p), C.POINTER(C.c_void_p), C.POINTER(C.c_void_p),
+                                     C.c_int32, C.c_void_p, C.c_int32, C.c_int32, C.c_int32, C.c_void_p]),
     "zdit_gemm_bf16": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int64, C.c_int64, C.c_int64,
                                  C.c_int64, C.c_void_p, C.c_void_p]),
     "zdit_patchify": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int32, C.c_int32, C.c_int32, C.c_void_p]),
@@ -261,6 +263,18 @@ def zdit_gemm_bf16(A, B, Cout, bias=None, stream=None):
     N = B.shape[0]
     _check(lib().zdit_gemm_bf16(_ptr(A), _ptr(B), _ptr(Cout), M, N, K, Cout.stride(0), _ptr(bias),
                                 _stream(stream)), "zdit_gemm_bf16")
+
+
+def zdit_adaln_project(w_ada, b_ada, out, temb, stream=None):
+    """out[i] [B, rows] = temb [B, E] . w_ada[i]^T [E, rows] + b_ada[i] for every i, one launch
+    (lists of device tensors: w_ada bf16 [rows, E], b_ada fp32 [rows] or None, out fp32 [B, rows])."""
+    n = len(w_ada)
+    rows, E = w_ada[0].shape
+    ws = (C.c_void_p * n)(*[t.data_ptr() for t in w_ada])
+    bs = (C.c_void_p * n)(*[(b.data_ptr() if b is not None else None) for b in b_ada])
+    os_ = (C.c_void_p * n)(*[t.data_ptr() for t in out])
+    _check(lib().zdit_adaln_project(ws, bs, os_, n, _ptr(temb), temb.shape[0], E, rows, _stream(stream)),
+           "zdit_adaln_project")
 
 
 def zdit_euler_cfg_step(x, v_pos, v_neg, g, sigma_cur, sigma_next, stream=None):

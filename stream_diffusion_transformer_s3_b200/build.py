@@ -2,7 +2,10 @@
 
 Each .cu file under csrc/ is compiled for sm_100a with nvcc, in parallel, then the
 objects are linked into a shared library next to this file.  Rebuilds only what is
-older than its sources.
+older than its sources, or everything when the compile flags changed.
+
+ZDIT_WAIT_LIMIT_MS in the environment sets the limit of the kernels' bounded waits
+(default 2000 ms; see include/zdit.h).
 """
 from __future__ import annotations
 
@@ -40,6 +43,17 @@ def _stale(target: str, deps) -> bool:
 def build(verbose: bool = False, extra_flags=()) -> str:
     os.makedirs(OBJ, exist_ok=True)
     nvcc = _nvcc()
+    extra_flags = list(extra_flags)
+    if os.environ.get("ZDIT_WAIT_LIMIT_MS"):
+        extra_flags.append(f"-DZDIT_WAIT_LIMIT_MS={int(os.environ['ZDIT_WAIT_LIMIT_MS'])}")
+    # objects built with other code-affecting flags are stale (-Xptxas -v only reports)
+    stamp = os.path.join(OBJ, "flags.txt")
+    code_flags = " ".join(f for f in extra_flags if f.startswith("-D"))
+    if not os.path.exists(stamp) or open(stamp).read() != code_flags:
+        for o in glob.glob(os.path.join(OBJ, "*.o")):
+            os.remove(o)
+        with open(stamp, "w") as fh:
+            fh.write(code_flags)
     headers = glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) + \
         glob.glob(os.path.join(ROOT, "include", "*.h"))
     sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")))

@@ -770,7 +770,8 @@ ZDIT_API zdit_status zdit_sigma_schedule(int32_t n_steps, float* sigmas) {
 ZDIT_API zdit_status zdit_rope_table(const int32_t* pos, int64_t T, int32_t head_dim, const int32_t rope_axes[3],
                                      float theta, float* cos_out, float* sin_out, void* stream) {
   if (!pos || !rope_axes || !cos_out || !sin_out || T < 0 || !(theta > 0.f)) return ZDIT_ERR_INVALID_ARG;
-  if (head_dim <= 0 || head_dim % 2 || rope_axes[0] + rope_axes[1] + rope_axes[2] != head_dim) return ZDIT_ERR_SHAPE;
+  if (head_dim <= 0 || head_dim % 2 || head_dim > 1024 || rope_axes[0] + rope_axes[1] + rope_axes[2] != head_dim)
+    return ZDIT_ERR_SHAPE;
   for (int i = 0; i < 3; ++i)
     if (rope_axes[i] < 0 || rope_axes[i] % 2) return ZDIT_ERR_SHAPE;
   if (T == 0) return ZDIT_OK;
@@ -793,6 +794,28 @@ ZDIT_API zdit_status zdit_joint_attention(const void* q, int32_t ldq, const void
   a.cu_seqlens_dev = varlen->cu_seqlens_dev; a.cu_seqlens_host = varlen->cu_seqlens_host;
   a.scale = 1.0f / sqrtf((float)head_dim);
   return launch_attention(a, static_cast<cudaStream_t>(stream));
+}
+
+ZDIT_API zdit_status zdit_adaln_project(const void* const* w_ada, const float* const* b_ada, float* const* out,
+                                        int32_t n_mat, const float* temb, int32_t batch, int32_t temb_dim,
+                                        int32_t rows, void* stream) {
+  if (!w_ada || !out || !temb) return ZDIT_ERR_INVALID_ARG;
+  if (n_mat <= 0 || n_mat > kMaxBlocks || batch <= 0 || batch > kMaxBatch || rows <= 0 || temb_dim <= 0 ||
+      temb_dim % 8 || temb_dim > 1024)
+    return ZDIT_ERR_SHAPE;
+  for (int i = 0; i < n_mat; ++i) {
+    if (!w_ada[i] || !out[i]) return ZDIT_ERR_INVALID_ARG;
+    if (!al16(w_ada[i]) || (reinterpret_cast<uintptr_t>(out[i]) & 3) ||
+        (b_ada && b_ada[i] && (reinterpret_cast<uintptr_t>(b_ada[i]) & 3)))
+      return ZDIT_ERR_ALIGNMENT;
+  }
+  if (!al16(temb)) return ZDIT_ERR_ALIGNMENT;
+  if (!device_ok()) return ZDIT_ERR_UNSUPPORTED;
+  const float* bias[kMaxBlocks];
+  for (int i = 0; i < n_mat; ++i) bias[i] = b_ada ? b_ada[i] : nullptr;
+  launch_gemv_batched(reinterpret_cast<const __nv_bfloat16* const*>(w_ada), bias, out, n_mat, temb, batch, temb_dim,
+                      rows, static_cast<cudaStream_t>(stream));
+  return cudaGetLastError() == cudaSuccess ? ZDIT_OK : ZDIT_ERR_CUDA;
 }
 
 ZDIT_API zdit_status zdit_gemm_bf16(const void* A, const void* B, float* C, int64_t M, int64_t N, int64_t K,

@@ -10,7 +10,13 @@
 
 namespace zdit {
 
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: no legal wait is near this
+// The limit of every bounded wait, set when the library is built (-DZDIT_WAIT_LIMIT_MS=...):
+// no wait of a healthy launch comes near the default 2 s, but a run slowed down from outside
+// (a profiler replaying kernels, a debugger) may need more.
+#ifndef ZDIT_WAIT_LIMIT_MS
+#define ZDIT_WAIT_LIMIT_MS 2000
+#endif
+constexpr uint64_t kWaitLimitNs = (uint64_t)(ZDIT_WAIT_LIMIT_MS) * 1000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

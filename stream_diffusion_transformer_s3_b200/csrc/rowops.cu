@@ -274,63 +274,104 @@ struct GemvBatch {
 };
 
 // Weight-streaming GEMV of the adaLN projections: out_m[b, r] = sum_e W_m[r, e] temb[b, e]
-// + bias_m[r].  A warp owns 8 rows and keeps their 16-byte weight loads in flight together
-// (the weights are read once, so the loads bypass L1); lane l covers columns [8l, 8l + 8)
-// of every 256-column chunk and holds the matching temb slice in registers.
+// + bias_m[r].  The rows of every matrix are cut into groups of 8; a warp reduces one group
+// at a time, lane l covering columns [8l, 8l + 8) of every 256-column chunk with the
+// matching temb slice.  The warps of a grid of a few CTAs per SM stride over all groups of
+// all matrices, and each loads the weights of its next (group, chunk) unit before reducing
+// the current one, so every warp keeps 8 16-byte loads in flight while it computes (the
+// weights are read once: the loads bypass L1).
 template <int B>
-__global__ void __launch_bounds__(128) adaln_gemv_kernel(const __grid_constant__ GemvBatch gb,
+__global__ void __launch_bounds__(128) adaln_gemv_kernel(const __grid_constant__ GemvBatch gb, int nm,
                                                          const float* __restrict__ temb, int E, int rows) {
-  const int m = blockIdx.y;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r0 = (blockIdx.x * 4 + warp) * 8;
-  if (r0 >= rows) return;
-  const __nv_bfloat16* W = gb.W[m];
+  const int lane = threadIdx.x & 31;
+  const int gpm = (rows + 7) / 8;              // groups per matrix
+  const int nch = (E + 255) / 256;             // 256-column chunks per row
+  const int64_t units_total = (int64_t)nm * gpm * nch;
+  const int64_t wstride = (int64_t)gridDim.x * (blockDim.x >> 5);
+  // unit k of this warp: group (gw + (k / nch) * wstride), chunk k % nch
+  const int64_t gw = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  auto load_unit = [&](int64_t grp, int ch, uint4 (&u)[8]) {
+    const int m = (int)(grp / gpm);
+    const int r0 = (int)(grp - (int64_t)m * gpm) * 8;
+    const int e0 = ch * 256 + lane * 8;
+    const __nv_bfloat16* W = gb.W[m];
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+      u[r] = (r0 + r < rows && e0 < E) ? __ldcs(reinterpret_cast<const uint4*>(W + (size_t)(r0 + r) * E + e0))
+                                       : make_uint4(0u, 0u, 0u, 0u);
+  };
+  if (gw * nch >= units_total) return;
+  uint4 cur[8], nxt[8];
+  load_unit(gw, 0, cur);
   float acc[8][B];
 #pragma unroll
   for (int r = 0; r < 8; ++r)
 #pragma unroll
     for (int b = 0; b < B; ++b) acc[r][b] = 0.f;
-  for (int e0 = lane * 8; e0 < E; e0 += 256) {
-    uint4 u[8];
-#pragma unroll
-    for (int r = 0; r < 8; ++r)
-      u[r] = r0 + r < rows ? __ldcs(reinterpret_cast<const uint4*>(W + (size_t)(r0 + r) * E + e0))
-                           : make_uint4(0u, 0u, 0u, 0u);
-    float t[B][8];
-#pragma unroll
-    for (int b = 0; b < B; ++b) {
-      const float4 lo = __ldg(reinterpret_cast<const float4*>(temb + (size_t)b * E + e0));
-      const float4 hi = __ldg(reinterpret_cast<const float4*>(temb + (size_t)b * E + e0 + 4));
-      t[b][0] = lo.x; t[b][1] = lo.y; t[b][2] = lo.z; t[b][3] = lo.w;
-      t[b][4] = hi.x; t[b][5] = hi.y; t[b][6] = hi.z; t[b][7] = hi.w;
+  for (int64_t grp = gw, ch = 0;;) {
+    // next unit of this warp
+    int64_t ngrp = grp;
+    int nchk = (int)ch + 1;
+    if (nchk == nch) {
+      nchk = 0;
+      ngrp = grp + wstride;
     }
+    const bool more = ngrp * nch < units_total;
+    if (more) load_unit(ngrp, nchk, nxt);
+    const int e0 = (int)ch * 256 + lane * 8;
+    if (e0 < E) {
+      float t[B][8];
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&u[r]);
+      for (int b = 0; b < B; ++b) {
+        const float4 lo = __ldg(reinterpret_cast<const float4*>(temb + (size_t)b * E + e0));
+        const float4 hi = __ldg(reinterpret_cast<const float4*>(temb + (size_t)b * E + e0 + 4));
+        t[b][0] = lo.x; t[b][1] = lo.y; t[b][2] = lo.z; t[b][3] = lo.w;
+        t[b][4] = hi.x; t[b][5] = hi.y; t[b][6] = hi.z; t[b][7] = hi.w;
+      }
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float w = __bfloat162float(h[j]);
+      for (int r = 0; r < 8; ++r) {
+        const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&cur[r]);
 #pragma unroll
-        for (int b = 0; b < B; ++b) acc[r][b] = fmaf(w, t[b][j], acc[r][b]);
+        for (int j = 0; j < 8; ++j) {
+          const float w = __bfloat162float(h[j]);
+#pragma unroll
+          for (int b = 0; b < B; ++b) acc[r][b] = fmaf(w, t[b][j], acc[r][b]);
+        }
       }
     }
-  }
-  const float* bias = gb.bias[m];
-  float* out = gb.out[m];
+    if (ch + 1 == nch) {
+      // the group's last chunk: reduce across the warp and store its 8 rows
+      const int m = (int)(grp / gpm);
+      const int r0 = (int)(grp - (int64_t)m * gpm) * 8;
+      const float* bias = gb.bias[m];
+      float* out = gb.out[m];
 #pragma unroll
-  for (int r = 0; r < 8; ++r) {
+      for (int r = 0; r < 8; ++r) {
 #pragma unroll
-    for (int b = 0; b < B; ++b) {
-      const float v = warp_sum(acc[r][b]);
-      if (lane == 0 && r0 + r < rows) out[(size_t)b * rows + r0 + r] = v + (bias != nullptr ? bias[r0 + r] : 0.f);
+        for (int b = 0; b < B; ++b) {
+          const float v = warp_sum(acc[r][b]);
+          acc[r][b] = 0.f;
+          if (lane == 0 && r0 + r < rows) out[(size_t)b * rows + r0 + r] = v + (bias != nullptr ? bias[r0 + r] : 0.f);
+        }
+      }
     }
+    if (!more) break;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) cur[r] = nxt[r];
+    grp = ngrp;
+    ch = nchk;
   }
 }
 
 template <int B>
 void launch_gemv_b(const GemvBatch& gb, int nm, const float* temb, int E, int rows, cudaStream_t s) {
-  dim3 grid((rows + 31) / 32, nm);
-  adaln_gemv_kernel<B><<<grid, 128, 0, s>>>(gb, temb, E, rows);
+  // 8 CTAs (32 warps) per SM at most; measured faster than a grid of only the resident
+  // CTAs (4 per SM at B = 2) with or without L2 prefetches ahead of the loads
+  const int64_t groups = (int64_t)nm * ((rows + 7) / 8);
+  int64_t ctas = (groups + 3) / 4;  // 4 warps per CTA, at least one group per warp
+  const int64_t cap = (int64_t)num_sms() * 8;
+  if (ctas > cap) ctas = cap;
+  adaln_gemv_kernel<B><<<(unsigned)ctas, 128, 0, s>>>(gb, nm, temb, E, rows);
 }
 
 void launch_gemv_any(const GemvBatch& gb, int nm, const float* temb, int B, int E, int rows, cudaStream_t s) {
@@ -369,24 +410,39 @@ __global__ void euler_cfg_kernel(float* __restrict__ x, const float* __restrict_
   }
 }
 
+// cos / sin of phi[t, i] = pos[t, axis(i)] * theta^(-2 j / width_axis) for a block of
+// kRopeTokens tokens per CTA: the frequencies of the pairs are computed once per CTA into
+// shared memory, then every (token, pair) angle and its cos / sin in double precision,
+// rounded to fp32 (the phases reach ~130 rad, so fp32 angles would be off by ~1e-5).
+constexpr int kRopeTokens = 32;
+
 __global__ void rope_table_kernel(const int* __restrict__ pos, int64_t T, int half_dim, int a0, int a1, int a2,
                                   double theta, float* __restrict__ cs, float* __restrict__ sn) {
-  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= T * half_dim) return;
-  const int64_t t = idx / half_dim;
-  const int i = (int)(idx % half_dim);
-  int axis, j, width;
-  if (i < a0 / 2) {
-    axis = 0; j = i; width = a0;
-  } else if (i < (a0 + a1) / 2) {
-    axis = 1; j = i - a0 / 2; width = a1;
-  } else {
-    axis = 2; j = i - (a0 + a1) / 2; width = a2;
+  extern __shared__ double omega[];  // [half_dim]
+  const int start1 = a0 / 2, start2 = (a0 + a1) / 2;  // first pair of axes 1 and 2
+  for (int i = threadIdx.x; i < half_dim; i += blockDim.x) {
+    int j, width;
+    if (i < a0 / 2) {
+      j = i; width = a0;
+    } else if (i < (a0 + a1) / 2) {
+      j = i - a0 / 2; width = a1;
+    } else {
+      j = i - (a0 + a1) / 2; width = a2;
+    }
+    omega[i] = pow(theta, -2.0 * j / width);
   }
-  const double omega = pow(theta, -2.0 * j / width);
-  const double phi = (double)pos[t * 3 + axis] * omega;
-  cs[idx] = (float)cos(phi);
-  sn[idx] = (float)sin(phi);
+  __syncthreads();
+  const int64_t t0 = (int64_t)blockIdx.x * kRopeTokens;
+  const int64_t n = (T - t0 < kRopeTokens ? T - t0 : kRopeTokens) * half_dim;
+  for (int64_t e = threadIdx.x; e < n; e += blockDim.x) {
+    const int64_t t = t0 + e / half_dim;
+    const int i = (int)(e % half_dim);
+    const int axis = i < start1 ? 0 : (i < start2 ? 1 : 2);
+    double s, c;
+    sincos((double)pos[t * 3 + axis] * omega[i], &s, &c);
+    cs[t * half_dim + i] = (float)c;
+    sn[t * half_dim + i] = (float)s;
+  }
 }
 
 struct TembParams {
@@ -599,10 +655,9 @@ void launch_euler_cfg(float* x, const float* vp, const float* vn, int64_t n, flo
 void launch_rope_table(const int* pos, int64_t T, int head_dim, const int* axes, float theta, float* cs, float* sn,
                        cudaStream_t s) {
   ProfScope ps(PROF_ROPE, 0.0, 8.0 * (double)T * (head_dim / 2) + 12.0 * T, s);
-  const int64_t n = T * (head_dim / 2);
-  if (n <= 0) return;
-  rope_table_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(pos, T, head_dim / 2, axes[0], axes[1], axes[2],
-                                                                 (double)theta, cs, sn);
+  if (T <= 0 || head_dim <= 0) return;
+  rope_table_kernel<<<(unsigned)((T + kRopeTokens - 1) / kRopeTokens), 256, (head_dim / 2) * sizeof(double), s>>>(
+      pos, T, head_dim / 2, axes[0], axes[1], axes[2], (double)theta, cs, sn);
 }
 
 void launch_timestep_embed(const float* t_host, int B, int E, float t_scale, const __nv_bfloat16* w1,

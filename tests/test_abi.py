@@ -127,3 +127,44 @@ def test_gate_up_interleave_layout():
     np.testing.assert_array_equal(g[128:256], w3[0:128])
     np.testing.assert_array_equal(g[256:384], w1[128:256])
     np.testing.assert_array_equal(g[384:512], w3[128:256])
+
+
+def test_static_block_checks_match_workspace_block_order():
+    # zdit_block_forward_static runs zdit_block_forward's checks, in the same order, before
+    # its own size check: a call that zdit_block_forward rejects for a bad pointer or shape
+    # is rejected with the same status, whatever its token count
+    L = Z.lib()
+    d = Z.Dims()
+    cfg = d.cfg(Z.flags_of())
+    w = Z.BlockWeights(**{f: _fake() for f, _ in Z.BlockWeights._fields_})
+    cu = (C.c_int32 * 3)(0, 1024, 2048)  # far more tokens than the static scratch holds
+    vl = Z.Varlen(2, _fake(), cu)
+    stat = lambda w_=w, x=_fake(), vl_=vl: L.zdit_block_forward_static(C.byref(cfg), C.byref(w_), C.byref(vl_), x,
+                                                                        _fake(), _fake(), _fake(), None)
+    full = lambda w_=w, x=_fake(), vl_=vl: L.zdit_block_forward(C.byref(cfg), C.byref(w_), C.byref(vl_), x, _fake(),
+                                                                 _fake(), _fake(), _fake(), 1 << 40, None)
+    assert stat(x=None) == full(x=None) == -1
+    assert stat(x=_fake((1 << 20) + 4)) == full(x=_fake((1 << 20) + 4)) == -3
+    w_nul = Z.BlockWeights(**{f: _fake() for f, _ in Z.BlockWeights._fields_})
+    w_nul.w_qkv = None
+    assert stat(w_=w_nul) == full(w_=w_nul) == -1
+    vl_bad = Z.Varlen(2, _fake(), (C.c_int32 * 3)(0, 1024, 1000))
+    assert stat(vl_=vl_bad) == full(vl_=vl_bad) == -2
+
+
+def test_adaln_project_rejects_bad_arguments_before_launch():
+    L = Z.lib()
+    arr = lambda *v: (C.c_void_p * len(v))(*v)
+    ws, bs, os_ = arr(1 << 20, 1 << 21), arr(1 << 22, None), arr(1 << 23, 1 << 24)
+    call = lambda w=ws, b=bs, o=os_, n=2, temb=_fake(), B=2, E=256, rows=15360: L.zdit_adaln_project(
+        w, b, o, n, temb, B, E, rows, None)
+    assert call(w=None) == -1
+    assert call(temb=None) == -1
+    assert call(w=arr(1 << 20, None)) == -1
+    assert call(n=0) == -2
+    assert call(B=9) == -2
+    assert call(E=100) == -2          # not a multiple of 8
+    assert call(E=2048) == -2         # wider than 1024
+    assert call(rows=0) == -2
+    assert call(w=arr(1 << 20, (1 << 21) + 8)) == -3   # weights must be 16-byte aligned
+    assert call(temb=_fake((1 << 20) + 4)) == -3

@@ -9,7 +9,7 @@ import torch
 import oracle as O
 import stream_diffusion_transformer_s3_b200 as Z
 from stream_diffusion_transformer_s3_b200 import synth
-from _gpu import bf16, dev, errors, host, require_gpu, rope_tables
+from _gpu import N_ROUND_ATTN, assert_parity, bf16, dev, host, require_gpu, rope_tables
 
 pytestmark = pytest.mark.gpu
 
@@ -42,8 +42,7 @@ def test_gemm_matches_float64_product(M, N, K):
     Z.zdit_gemm_bf16(bf16(A), bf16(B), out, bias=dev(bias))
     assert Z.zdit_device_status() == 0
     ref = A.astype(np.float64) @ B.astype(np.float64).T + bias
-    e = errors(host(out), ref)
-    assert e["rel_l2"] < gemm_tol(K), e
+    assert_parity(host(out), ref, gemm_tol(K), rtol=gemm_tol(K), label=f"gemm {M}x{N}x{K}")
 
 
 def test_gemm_large_k_and_many_tiles():
@@ -56,8 +55,33 @@ def test_gemm_large_k_and_many_tiles():
     Z.zdit_gemm_bf16(bf16(A), bf16(B), out)
     assert Z.zdit_device_status() == 0
     ref = A.astype(np.float64) @ B.astype(np.float64).T
-    e = errors(host(out), ref)
-    assert e["rel_l2"] < gemm_tol(K), e
+    assert_parity(host(out), ref, gemm_tol(K), rtol=gemm_tol(K), label=f"gemm {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("n_mat,B,rows,E", [
+    (3, 2, 4 * 3840, 256),   # three blocks' adaLN projections at full width, cond/uncond
+    (45, 8, 4 * 256, 256),   # more matrices than one launch holds, the largest batch
+    (2, 1, 77, 1024),        # ragged rows (groups of 8 cut), four 256-column chunks
+])
+def test_adaln_project_matches_oracle(n_mat, B, rows, E):
+    temb = synth.randn(8, 900, (B, E))
+    ws = [synth.bf16_round(synth.randn(8, 901 + i, (rows, E), 0.02)) for i in range(n_mat)]
+    bs = [synth.randn(8, 1001 + i, (rows,), 0.02) if i % 2 == 0 else None for i in range(n_mat)]
+    outs = [torch.full((B, rows), float("nan"), device="cuda") for _ in range(n_mat)]
+    Z.zdit_adaln_project([bf16(w) for w in ws], [dev(b) if b is not None else None for b in bs], outs, dev(temb))
+    assert Z.zdit_device_status() == 0
+    tol = 3.0 * np.sqrt(E) * 2.0 ** -23
+    refs = []
+    for i in range(n_mat):
+        if rows % 4 == 0 and bs[i] is not None:
+            # the oracle's adaLN step: four chunks (scale_attn, gate_attn, scale_ffn, gate_ffn)
+            refs.append(np.concatenate(O.adaln_vectors(temb, {"w_ada": ws[i], "b_ada": bs[i]}, rows // 4, O.Flags()),
+                                       axis=1))
+        else:
+            refs.append(temb.astype(np.float64) @ ws[i].astype(np.float64).T + (0.0 if bs[i] is None else bs[i]))
+    # rows of the check: (matrix, branch)
+    assert_parity(np.concatenate([host(o) for o in outs]), np.concatenate(refs), tol, rtol=tol,
+                  label=f"adaLN projections, {n_mat} matrices x {B} branches x {rows}")
 
 
 def _attn_case(lengths, H, seed=0):
@@ -82,8 +106,7 @@ def test_attention_matches_oracle(lengths, H):
     Z.zdit_joint_attention(bf16(c["q"]), bf16(c["k"]), bf16(c["v"]), o, vl, H)
     assert Z.zdit_device_status() == 0
     ref = O.joint_attention(q, k, v, c["cu_seqlens"]).reshape(T, H * 128)
-    e = errors(host(o), ref)
-    assert e["rel_l2"] < 1e-2, e
+    assert_parity(host(o), ref, 1e-2, n_round=N_ROUND_ATTN, label=f"attention {lengths} x {H}")
 
 
 def test_attention_full_width_config5_small():
@@ -96,8 +119,7 @@ def test_attention_full_width_config5_small():
     Z.zdit_joint_attention(bf16(c["q"]), bf16(c["k"]), bf16(c["v"]), o, vl, 30)
     assert Z.zdit_device_status() == 0
     ref = O.joint_attention(q, k, v, c["cu_seqlens"]).reshape(T, -1)
-    e = errors(host(o), ref)
-    assert e["rel_l2"] < 1e-2, e
+    assert_parity(host(o), ref, 1e-2, n_round=N_ROUND_ATTN, label="attention 1152/1056 x 30")
 
 
 def test_attention_large_logits_move_reference_max():
@@ -113,7 +135,7 @@ def test_attention_large_logits_move_reference_max():
     Z.zdit_joint_attention(bf16(q.reshape(L, -1)), bf16(k.reshape(L, -1)), bf16(v.reshape(L, -1)), o, vl, 1)
     assert Z.zdit_device_status() == 0
     ref = O.joint_attention(q, k, v, np.array([0, L])).reshape(L, -1)
-    assert errors(host(o), ref)["rel_l2"] < 1e-2
+    assert_parity(host(o), ref, 1e-2, n_round=N_ROUND_ATTN, label="attention, moving max")
 
 
 def test_rope_table_matches_oracle():
