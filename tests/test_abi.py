@@ -168,3 +168,13 @@ def test_adaln_project_rejects_bad_arguments_before_launch():
     assert call(rows=0) == -2
     assert call(w=arr(1 << 20, (1 << 21) + 8)) == -3   # weights must be 16-byte aligned
     assert call(temb=_fake((1 << 20) + 4)) == -3
+
+
+def test_rope_table_rejects_bad_widths_before_launch():
+    L = Z.lib()
+    axes = lambda a, b, c: (C.c_int32 * 3)(a, b, c)
+    call = lambda hd, ax: L.zdit_rope_table(_fake(), 16, hd, ax, 10000.0, _fake(), _fake(), None)
+    assert call(128, axes(32, 48, 50)) == -2       # axes do not add up to the head width
+    assert call(127, axes(31, 48, 48)) == -2       # odd head width
+    assert call(2048, axes(512, 768, 768)) == -2   # wider than the 1024 the tables support
+    assert L.zdit_rope_table(None, 16, 128, axes(32, 48, 48), 10000.0, _fake(), _fake(), None) == -1

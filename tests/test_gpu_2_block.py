@@ -79,3 +79,20 @@ def test_band_overlap_is_bitwise_neutral():
     finally:
         Z.zdit_profile_end()
     assert np.array_equal(banded, serial)
+
+
+@pytest.mark.parametrize("flags", [O.Flags(tanh_gate=True), O.Flags(qk_norm=True)])
+def test_config2_full_width_block_other_flags(flags):
+    # full width with the tanh gate, and QK-norm with the sandwich norm on
+    case = synth.block_case(3, synth.FULL, 16, 16, [64, 32], [45, 1], x_max=6.7e3, qk_norm=flags.qk_norm)
+    _check(case, synth.FULL, flags)
+
+
+@pytest.mark.parametrize("n_heads,ffn", [(12, 512), (64, 256)])
+def test_block_widths_of_every_row_kernel_instance(n_heads, ffn):
+    # the row kernels keep a whole row in registers in 1, 2, 4 or 8 float4 per thread: width 1536
+    # (12 heads) takes the 2-vector instance, width 8192 (64 heads, the widest the library accepts)
+    # the 8-vector one; the others run in every test above (widths 256 and 3840)
+    d = synth.BlockDims(dim=128 * n_heads, n_heads=n_heads, head_dim=128, ffn_hidden=ffn)
+    case = synth.block_case(5, d, 8, 8, [64, 32], [40, 1])
+    _check(case, d, O.Flags())

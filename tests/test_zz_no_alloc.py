@@ -5,10 +5,12 @@ own pool, or a loop that must not pay cudaMalloc's device-wide synchronization).
 Checks, through the C ABI on the GPU, that two calls in a row (sharing the library's
 static scratch) give the same block output as zdit_block_forward with a caller
 workspace, within the block-parity tolerance; that those two calls leave the device's
-free memory unchanged (they allocate nothing); and that a call too large for the 40 MiB
-scratch is refused before any launch.  This file is collected last."""
+free memory unchanged (they allocate nothing); that a call of the most tokens the 40 MiB
+scratch admits matches the workspace path too; and that a call too large for the scratch is
+refused before any launch.  This file is collected last."""
 import ctypes as C
 
+import numpy as np
 import pytest
 import torch
 
@@ -72,3 +74,30 @@ def test_static_scratch_refuses_oversized_call():
     code = Z.lib().zdit_block_forward_static(C.byref(cfg), C.byref(wts), C.byref(vl.struct), C.c_void_p(1 << 20),
                                              C.c_void_p(1 << 20), C.c_void_p(1 << 20), C.c_void_p(1 << 20), None)
     assert code == -4  # ZDIT_ERR_WORKSPACE, nothing launched
+
+
+def test_static_scratch_at_its_largest_admitted_size():
+    # the most tokens whose workspace still fits the 40 MiB scratch at full width, in two branches
+    dims = Z.Dims()
+    fl = Z.flags_of()
+    T = max(t for t in range(600, 1200) if Z.block_workspace_bytes(dims, fl, t, 2) <= (40 << 20))
+    assert Z.block_workspace_bytes(dims, fl, T + 1, 2) > (40 << 20)
+    d = synth.FULL
+    n_img = 16 * 16
+    lens = [T // 2, T - T // 2]
+    rng = np.random.default_rng(0)
+    x0 = (rng.standard_normal((T, d.dim)) * 3.0).astype(np.float32)
+    cu = synth.cu_seqlens(lens)
+    pos = np.concatenate([synth.branch_positions(16, 16, L - n_img)[:L] if L > n_img else
+                          synth.branch_positions(16, 16, 0)[:L] for L in lens]).astype(np.int32)
+    w = Z.DeviceBlock(synth.block_weights(0, 0, d))
+    vl = Z.DeviceVarlen(cu)
+    temb = dev(synth.randn(0, 9, (2, d.temb_dim)))
+    cs, sn = rope_tables(pos, dims)
+    x_ref = dev(x0)
+    ws = torch.empty(Z.block_workspace_bytes(dims, fl, T, 2), dtype=torch.uint8, device="cuda")
+    Z.zdit_block_forward(dims, fl, w, vl, x_ref, temb, cs, sn, ws)
+    x = dev(x0)
+    Z.zdit_block_forward_static(dims, fl, w, vl, x, temb, cs, sn)
+    assert Z.zdit_device_status() == 0
+    assert_parity(host(x), host(x_ref), TOL, base=x0, n_round=N_ROUND_BLOCK, label=f"static scratch, {T} tokens")
