@@ -60,6 +60,13 @@ def forward_flops() -> float:
 NCU_TRAFFIC = {"kernel": "gemm_gate_up_swiglu", "bytes": 409473536 + 156275456, "src_hash": "b057c4233dacc1b0"}
 
 
+# What bounds each kernel kind of the library's profiler (its `kernels` table).
+KERNEL_BOUND = {"gemm_qkv_rope": "tensor", "gemm_out_proj": "tensor", "gemm_gate_up_swiglu": "tensor",
+                "gemm_down_proj": "tensor", "attention": "tensor", "residual_norm": "hbm",
+                "norm_modulate": "hbm", "adaln_gemv": "hbm", "euler_cfg": "hbm",
+                "gemm_embed_final": "latency", "rope_table": "latency", "misc": "latency"}
+
+
 def gemm_src_hash() -> str:
     import hashlib
     h = hashlib.sha256()
@@ -444,6 +451,14 @@ def run_ours(args):
             row["tflops"] = round(k["flops"] / (k["total_ms"] * 1e-3) / 1e12, 1)
         if k["bytes"] > 0:
             row["gbs"] = round(k["bytes"] / (k["total_ms"] * 1e-3) / 1e9, 1)
+        # the bound of each kernel kind and its fraction of the matching measured peak (the
+        # projections' and attention's bf16 peak as above; the row kernels' copy bandwidth)
+        if n in KERNEL_BOUND:
+            row["bound"] = KERNEL_BOUND[n]
+            if KERNEL_BOUND[n] == "tensor" and "tflops" in row:
+                row["frac"] = round(row["tflops"] / peak, 4)
+            elif KERNEL_BOUND[n] == "hbm" and "gbs" in row:
+                row["frac"] = round(row["gbs"] / peaks["hbm_gbs"], 4)
         kern_summary[n] = row
 
     if rank == 0:

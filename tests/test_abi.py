@@ -178,3 +178,19 @@ def test_rope_table_rejects_bad_widths_before_launch():
     assert call(127, axes(31, 48, 48)) == -2       # odd head width
     assert call(2048, axes(512, 768, 768)) == -2   # wider than the 1024 the tables support
     assert L.zdit_rope_table(None, 16, 128, axes(32, 48, 48), 10000.0, _fake(), _fake(), None) == -1
+
+
+def test_bench_names_a_bound_for_every_profiled_kernel_kind():
+    # bench.py reports each kernel kind's fraction of the peak of its bound; every kind the
+    # library's profiler records (the name table in prof.cu) must have one
+    import re as _re
+    import sys as _sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    _sys.path.insert(0, root)
+    import bench
+    src = open(os.path.join(root, "stream_diffusion_transformer_s3_b200", "csrc", "prof.cu")).read()
+    table = src[src.index("{", src.index("const char*")):src.index("};", src.index("const char*"))]
+    kinds = _re.findall(r'"(\w+)"', table)
+    assert len(kinds) == 12
+    assert set(kinds) == set(bench.KERNEL_BOUND)
+    assert set(bench.KERNEL_BOUND.values()) <= {"tensor", "hbm", "latency"}
