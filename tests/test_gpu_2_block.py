@@ -96,3 +96,9 @@ def test_block_widths_of_every_row_kernel_instance(n_heads, ffn):
     d = synth.BlockDims(dim=128 * n_heads, n_heads=n_heads, head_dim=128, ffn_hidden=ffn)
     case = synth.block_case(5, d, 8, 8, [64, 32], [40, 1])
     _check(case, d, O.Flags())
+
+
+def test_full_width_single_branch_odd_length():
+    # one branch of 333 tokens (256 image + 77 caption rows): no multiple of the 128-row tiles
+    case = synth.block_case(6, synth.FULL, 16, 16, [77], [50], x_max=6.7e3)
+    _check(case, synth.FULL, O.Flags())

@@ -50,3 +50,14 @@ def test_full_width_full_depth_stack_256px():
     got = run_stack(W, case, d, 2, 2, 30, 2560, blocks=src.device)
     # per-block bound 2e-2; the measured 34-block free-running error is 4.9e-3
     assert_parity(got, ref, 2e-2, n_round=N_ROUND_BLOCK, label="stack full width, 34 blocks")
+
+
+def test_small_stack_three_branches():
+    # three branches (e.g. two prompts and the empty one) in one call: the layout kernel, the
+    # adaLN projections and the varlen attention over three segments
+    d = synth.BlockDims(dim=256, n_heads=2, head_dim=128, ffn_hidden=384)
+    W = synth.stack_weights(8, d, n_noise=1, n_context=1, n_main=2, cap_dim=128)
+    case = synth.stack_case(8, 8, 8, [64, 32, 96], [45, 1, 70], [0.3, 0.3, 0.7], cap_dim=128)
+    got = run_stack(W, case, d, 1, 1, 2, 128)
+    ref = O.stack_forward(case, W, d)
+    assert_parity(got, ref, 2e-2, n_round=N_ROUND_BLOCK, label="stack, three branches")
