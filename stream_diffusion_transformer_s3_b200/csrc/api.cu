@@ -34,15 +34,12 @@ void launch_stack_layout(const int* n_cap, int B, int grid_h, int grid_w, int* p
 
 zdit_status read_and_clear_device_error();
 
+// SM count of the current device (queried per call: a process may drive several devices)
 int num_sms() {
-  static int n = 0;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  });
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      n <= 0)
+    n = 148;
   return n;
 }
 
@@ -51,17 +48,11 @@ namespace {
 constexpr int kMaxBatch = 8;
 constexpr int kMaxBlocks = 256;
 
+// the current device is a compute capability 10.x part (checked per call, like num_sms)
 bool device_ok() {
-  static int ok = -1;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    int dev = 0, major = 0;
-    ok = (cudaGetDevice(&dev) == cudaSuccess &&
-          cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) == cudaSuccess && major == 10)
-             ? 1
-             : 0;
-  });
-  return ok == 1;
+  int dev = 0, major = 0;
+  return cudaGetDevice(&dev) == cudaSuccess &&
+         cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) == cudaSuccess && major == 10;
 }
 
 size_t align_up(size_t v, size_t a = 256) { return (v + a - 1) / a * a; }

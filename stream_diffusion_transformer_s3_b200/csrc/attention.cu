@@ -418,12 +418,9 @@ zdit_status launch_attention(const AttnArgs& a, cudaStream_t s) {
   if (!make_tmap_bf16_2d(&tq, a.q, a.T, cols, a.ldq, TILE, 64)) return ZDIT_ERR_CUDA;
   if (!make_tmap_bf16_2d(&tk, a.k, a.T, cols, a.ldk, TILE, 64)) return ZDIT_ERR_CUDA;
   if (!make_tmap_bf16_2d(&tv, a.v, a.T, cols, a.ldv, TILE, 64)) return ZDIT_ERR_CUDA;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
-      return ZDIT_ERR_CUDA;
-    attr = true;
-  }
+  // per launch: the opt-in belongs to the current context (see launch_epi)
+  if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
+    return ZDIT_ERR_CUDA;
   AParams p;
   p.ldo = a.ldo;
   p.n_heads = a.n_heads;

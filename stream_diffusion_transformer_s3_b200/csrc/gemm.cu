@@ -582,24 +582,19 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 template <int EPI>
 zdit_status launch_epi(const CUtensorMap& ta, const CUtensorMap& tb, const KParams& kp, int grid, bool pair,
                        cudaStream_t s) {
-  static bool attr_set = false, attr_pair_set = false;
+  // The shared-memory opt-in is a property of the current context: set on every launch
+  // (cheap, and legal inside stream capture) so a second device, or a context created
+  // again after a reset, never launches without it.
   if (pair) {
-    if (!attr_pair_set) {
-      if (cudaFuncSetAttribute(gemm_pair_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               PairRing<pair_bk<EPI>()>::SMEM_BYTES) !=
-          cudaSuccess)
-        return ZDIT_ERR_CUDA;
-      attr_pair_set = true;
-    }
+    if (cudaFuncSetAttribute(gemm_pair_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             PairRing<pair_bk<EPI>()>::SMEM_BYTES) != cudaSuccess)
+      return ZDIT_ERR_CUDA;
     launch_dependent(gemm_pair_kernel<EPI>, dim3(grid), dim3(THREADS), PairRing<pair_bk<EPI>()>::SMEM_BYTES, s, ta, tb,
                      kp);
   } else {
-    if (!attr_set) {
-      if (cudaFuncSetAttribute(gemm_tc_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
-          cudaSuccess)
-        return ZDIT_ERR_CUDA;
-      attr_set = true;
-    }
+    if (cudaFuncSetAttribute(gemm_tc_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
+        cudaSuccess)
+      return ZDIT_ERR_CUDA;
     launch_dependent(gemm_tc_kernel<EPI>, dim3(grid), dim3(THREADS), SMEM_BYTES, s, ta, tb, kp);
   }
   return cudaGetLastError() == cudaSuccess ? ZDIT_OK : ZDIT_ERR_CUDA;

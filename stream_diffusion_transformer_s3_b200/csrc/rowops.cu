@@ -25,16 +25,11 @@ namespace zdit {
 // parameter; zdit_device_status reads and clears it.
 __device__ int g_device_error = 0;
 
+// Looked up on every call, not cached: the address belongs to the current device's
+// context and changes when that context is destroyed and created again.
 int* device_error_ptr() {
-  static int* ptrs[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) return nullptr;
-  if (ptrs[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_device_error) == cudaSuccess) ptrs[dev] = static_cast<int*>(p);
-  }
-  return ptrs[dev];
+  void* p = nullptr;
+  return cudaGetSymbolAddress(&p, g_device_error) == cudaSuccess ? static_cast<int*>(p) : nullptr;
 }
 
 zdit_status read_and_clear_device_error() {
