@@ -57,6 +57,9 @@ def forward_flops() -> float:
 # x 3840), from one ncu capture of that kernel (dram__bytes_read.sum + dram__bytes_write.sum),
 # valid for the GEMM sources with this hash only; any change to them makes the figure stale
 # (reported null).
+# The headline metric, shared by this implementation's line and the reference arm's.
+METRIC = "DiT forward TFLOP/s (1024^2, 34-block step, bf16, 1 B200)"
+
 NCU_TRAFFIC = {"kernel": "gemm_gate_up_swiglu", "bytes": 402328576 + 155948288, "src_hash": "d230e725b4f8169d"}
 
 
@@ -463,7 +466,7 @@ def run_ours(args):
 
     if rank == 0:
         res = {
-            "metric": "DiT forward TFLOP/s (1024^2, 34-block step, bf16, 1 B200)",
+            "metric": METRIC,
             "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
@@ -617,7 +620,7 @@ def run_reference(args):
     value = flops / sec / 1e12
     sample = ("each step: one full-width main block of the workload on its uncond branch (L=4128 tokens), "
               "NumPy float64 oracle on the host cores")
-    res = {"metric": "DiT forward TFLOP/s (1024^2, 34-block step, bf16, 1 B200)", "impl": "reference",
+    res = {"metric": METRIC, "impl": "reference",
            "value": round(value, 5), "unit": "TFLOP/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sec * 1e3, 1),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
