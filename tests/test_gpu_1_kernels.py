@@ -160,6 +160,17 @@ def test_euler_cfg_matches_oracle(n, g, with_neg):
     np.testing.assert_allclose(host(x), ref, rtol=1e-6, atol=1e-6)
 
 
+def test_patchify_round_trip_non_square_latent():
+    # 12 x 20 latent -> 6 x 10 token grid: a swapped height and width would reorder the tokens
+    lat = synth.randn(43, 11, (16, 12, 20))
+    t = torch.empty(6 * 10, 64, device="cuda")
+    Z.zdit_patchify(dev(lat), t)
+    np.testing.assert_array_equal(host(t), O.patchify(lat))
+    back = torch.empty(16, 12, 20, device="cuda")
+    Z.zdit_unpatchify(t, back)
+    np.testing.assert_array_equal(host(back), lat)
+
+
 def test_patchify_round_trip_matches_oracle():
     lat = synth.randn(42, 11, (16, 128, 128))
     t = torch.empty(64 * 64, 64, device="cuda")

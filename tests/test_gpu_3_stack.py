@@ -61,3 +61,15 @@ def test_small_stack_three_branches():
     got = run_stack(W, case, d, 1, 1, 2, 128)
     ref = O.stack_forward(case, W, d)
     assert_parity(got, ref, 2e-2, n_round=N_ROUND_BLOCK, label="stack, three branches")
+
+
+def test_small_stack_non_square_grid():
+    # a 6 x 16 image grid (the stack takes image-token counts that are multiples of 32): the
+    # image positions (h, w) and their RoPE axes, the patch-token order and the final layer's
+    # image rows must all follow height and width, not a square
+    d = synth.BlockDims(dim=256, n_heads=2, head_dim=128, ffn_hidden=384)
+    W = synth.stack_weights(10, d, n_noise=1, n_context=1, n_main=2, cap_dim=128)
+    case = synth.stack_case(10, 6, 16, [64, 32], [45, 1], [0.5, 0.5], cap_dim=128)
+    got = run_stack(W, case, d, 1, 1, 2, 128)
+    ref = O.stack_forward(case, W, d)
+    assert_parity(got, ref, 2e-2, n_round=N_ROUND_BLOCK, label="stack, 6 x 16 grid")

@@ -76,6 +76,22 @@ def test_sample_entry_point_matches_oracle(dedup):
     _check(host(lat), ref, f"zdit_sample dedup={dedup}")
 
 
+def test_sample_non_square_latent():
+    # latent 16 x 12 x 32 (6 x 16 patch grid) through the whole-image entry point
+    d, W, _, caps = _small_setup()
+    latent = synth.latent_noise(44, (16, 12, 32))
+    stack = Z.DeviceStack(W, dims_of(d), 2, 2, 2, patch_dim=64, cap_dim=128)
+    call = Z.StackCall((6, 16), [64, 32], [45, 1], [0.0, 0.0], dev(caps), dev(caps))
+    ws = torch.empty(Z.sample_workspace_bytes(stack, call), dtype=torch.uint8, device="cuda")
+    lat = dev(latent)
+    Z.zdit_sample(stack, call, lat, ws, n_steps=8, guidance=1.0)
+    assert Z.zdit_device_status() == 0
+    cond = {"caps": caps[:45], "n_cap": 64, "n_valid": 45}
+    unc = {"caps": caps[45:], "n_cap": 32, "n_valid": 1}
+    ref = O.sample(latent, cond, unc, W, d, g=1.0, n_steps=8)
+    _check(host(lat), ref, "zdit_sample, 6 x 16 grid")
+
+
 def test_sample_single_branch_guidance_zero():
     d, W, latent, caps = _small_setup()
     stack = Z.DeviceStack(W, dims_of(d), 2, 2, 2, patch_dim=64, cap_dim=128)
