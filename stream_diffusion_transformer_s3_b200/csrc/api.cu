@@ -1,6 +1,7 @@
 // C-ABI entry points: host-side validation, workspace carving and the launch
 // sequence of the block, the stack and the sampler update.  No compute happens here;
 // every step runs in the kernels of gemm.cu, attention.cu and rowops.cu.
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -634,14 +635,44 @@ zdit_status sample_run(const zdit_stack_cfg* cfg, const zdit_stack_weights* w, c
   return cudaGetLastError() == cudaSuccess ? ZDIT_OK : ZDIT_ERR_CUDA;
 }
 
+// Unique id of the current CUDA context (cuCtxGetId: ids are never reused within a
+// process), 0 when it cannot be read.  Handles cached across calls (the sampler's graph and
+// capture stream) belong to one context and are not reused after it is destroyed and
+// created again.
+unsigned long long current_context_id() {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrent>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetId>(p);
+  });
+  CUcontext c = nullptr;
+  unsigned long long id = 0;
+  if (get_current == nullptr || get_id == nullptr || get_current(&c) != CUDA_SUCCESS || c == nullptr ||
+      get_id(c, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
 // One cached executable graph of the sampler (zdit_sample_cfg.use_graph).
 struct SampleGraph {
   std::mutex mu;
   std::vector<uint8_t> key;
   cudaGraphExec_t exec = nullptr;
+  unsigned long long exec_context = 0;  // context the graph belongs to
   int64_t launches = 0;
   cudaStream_t capture_stream = nullptr;
-  int capture_device = -1;
+  unsigned long long stream_context = 0;  // context the capture stream belongs to
 };
 
 SampleGraph& sample_graph() {
@@ -690,9 +721,10 @@ ZDIT_API zdit_status zdit_sample(const zdit_stack_cfg* cfg, const zdit_stack_wei
     const uint8_t* b = static_cast<const uint8_t*>(p);
     key.insert(key.end(), b, b + n);
   };
-  int dev = 0;
-  cudaGetDevice(&dev);
-  put(&dev, sizeof(dev));
+  // the context, not only the device: after a context is destroyed its graph is not reused
+  const unsigned long long ctx = current_context_id();
+  if (ctx == 0) return sample_run(cfg, w, in, sc, latent, workspace, d, in2, t_host, s);
+  put(&ctx, sizeof(ctx));
   put(cfg, sizeof(*cfg));
   put(w, sizeof(*w));
   put(w->blocks, sizeof(zdit_block_weights) * (size_t)(cfg->n_noise_refiner + cfg->n_context_refiner + cfg->n_main));
@@ -711,9 +743,13 @@ ZDIT_API zdit_status zdit_sample(const zdit_stack_cfg* cfg, const zdit_stack_wei
   if (g.exec == nullptr || g.key != key) {
     // capture on a private stream (the caller's may be the legacy default stream, which
     // cannot capture); nothing runs during capture, the graph is then launched on `s`
-    if (g.capture_stream == nullptr || g.capture_device != dev) {
-      if (cudaStreamCreateWithFlags(&g.capture_stream, cudaStreamNonBlocking) != cudaSuccess) return ZDIT_ERR_CUDA;
-      g.capture_device = dev;
+    if (g.capture_stream == nullptr || g.stream_context != ctx) {
+      // a stream of another context is left alone: it may no longer exist
+      if (cudaStreamCreateWithFlags(&g.capture_stream, cudaStreamNonBlocking) != cudaSuccess) {
+        g.capture_stream = nullptr;
+        return ZDIT_ERR_CUDA;
+      }
+      g.stream_context = ctx;
     }
     cudaStream_t cs = g.capture_stream;
     const int64_t before = zdit_launch_count();
@@ -729,8 +765,9 @@ ZDIT_API zdit_status zdit_sample(const zdit_stack_cfg* cfg, const zdit_stack_wei
     const cudaError_t ie = cudaGraphInstantiate(&exec, graph, 0);
     cudaGraphDestroy(graph);
     if (ie != cudaSuccess) return ZDIT_ERR_CUDA;
-    if (g.exec != nullptr) cudaGraphExecDestroy(g.exec);
+    if (g.exec != nullptr && g.exec_context == ctx) cudaGraphExecDestroy(g.exec);
     g.exec = exec;
+    g.exec_context = ctx;
     g.key = key;
     g.launches = zdit_launch_count() - before;  // counted once at capture, once per replay below
     return cudaGraphLaunch(g.exec, s) == cudaSuccess ? ZDIT_OK : ZDIT_ERR_CUDA;
