@@ -281,8 +281,11 @@ typedef struct {
   int32_t dedup_noise;    /* 1: noise refiner computed once for branches  */
   int32_t use_graph;      /* 1: the whole launch sequence is captured as one CUDA graph
                              on the first call and replayed while every argument (pointers,
-                             sizes, steps, guidance, device) stays the same; not used while
-                             the profiler records.  The library keeps one such graph. */
+                             sizes, steps, guidance) and the CUDA context stay the same (a
+                             context created again captures afresh); not used while the
+                             profiler records, nor when the context's id cannot be read
+                             (the launches then run directly).  The library keeps one such
+                             graph. */
 } zdit_sample_cfg;
 
 /* in: batch 1 or 2, grid, n_cap, n_valid, cap_feats as for zdit_stack_forward;
